@@ -1,0 +1,91 @@
+"""The pins must catch plausible slips in the oracle (CPU only).
+
+Each case compiles a copy of the oracle's C source with one planted mistake
+into a temporary directory, swaps it in for the real library, and checks that
+at least one pin of `test_oracle_pins.py` fails.  The real oracle is put
+back afterwards.
+"""
+import ctypes
+import inspect
+import json
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
+
+WRITE_LINE = "row[j] = a * (row[j] - e * ki * p[j]) + w * ki * v[j];"
+CAUSAL_BODY = """            transition(S, p, J->k + tok * dk, J->v + tok * dv, J->alpha[tok],
+                       J->erase[tok], J->write[tok], dk, dv);
+            readout(S, J->q + tok * dk, dk, dv, J->o + tok * dv, 0);"""
+REVERSE_BODY = """            readout(S, J->q + tok * dk, dk, dv, J->o + tok * dv, acc);
+            transition(S, p, J->k + tok * dk, J->v + tok * dv, J->alpha[tok],
+                       J->erase[tok], J->write[tok], dk, dv);"""
+
+MUTATIONS = {
+    "erase_dropped": (WRITE_LINE, "row[j] = a * (row[j]) + w * ki * v[j];"),
+    "erase_sign_flipped": (WRITE_LINE, "row[j] = a * (row[j] + e * ki * p[j]) + w * ki * v[j];"),
+    "alpha_on_write": (WRITE_LINE, "row[j] = a * (row[j] - e * ki * p[j] + w * ki * v[j]);"),
+    "alpha_dropped": (WRITE_LINE, "row[j] = (row[j] - e * ki * p[j]) + w * ki * v[j];"),
+    "write_dropped": (WRITE_LINE, "row[j] = a * (row[j] - e * ki * p[j]);"),
+    "erase_uses_alpha_twice": (WRITE_LINE, "row[j] = a * (row[j] - a * e * ki * p[j]) + w * ki * v[j];"),
+    "causal_readout_before_write": (CAUSAL_BODY, """            readout(S, J->q + tok * dk, dk, dv, J->o + tok * dv, 0);
+            transition(S, p, J->k + tok * dk, J->v + tok * dv, J->alpha[tok],
+                       J->erase[tok], J->write[tok], dk, dv);"""),
+    "reverse_readout_after_write": (REVERSE_BODY, """            transition(S, p, J->k + tok * dk, J->v + tok * dv, J->alpha[tok],
+                       J->erase[tok], J->write[tok], dk, dv);
+            readout(S, J->q + tok * dk, dk, dv, J->o + tok * dv, acc);"""),
+    "readout_transposed_state": ("acc += S[(size_t)i * dv + j] * q[i];",
+                                 "acc += S[(size_t)j * dk + i] * q[i];"),
+    "erase_projects_query": ("for (int i = 0; i < dk; ++i) acc += S[(size_t)i * dv + j] * k[i];\n        p[j] = acc;",
+                             "for (int i = 0; i < dk; ++i) acc += S[(size_t)i * dv + j] * k[0];\n        p[j] = acc;"),
+    "state_in_ignored": ("if (J->s_fwd0) memcpy(S, J->s_fwd0", "if (0) memcpy(S, J->s_fwd0"),
+    "bidir_overwrites_causal": ("const int acc = (J->mode == 2);", "const int acc = 0;"),
+}
+
+
+def _pin_functions():
+    out = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        if name == "test_worked_examples":
+            for ex in pins._golden():
+                out.append((name + "[" + ex["name"] + "]", lambda ex=ex: pins.test_worked_examples(ex)))
+        elif name == "test_split_calls_equal_one_call":
+            out.append((name, lambda: pins.test_split_calls_equal_one_call(17)))
+        else:
+            out.append((name, fn))
+    return out
+
+
+@pytest.mark.parametrize("mutation", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(mutation, tmp_path):
+    old, new = MUTATIONS[mutation]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, "mutation anchor not found: %s" % mutation
+    mutated = src.replace(old, new)
+    c_path = tmp_path / "mut.c"
+    so_path = tmp_path / "libmut.so"
+    c_path.write_text(mutated)
+    subprocess.check_call(["gcc", "-O1", "-std=c99", "-fPIC", "-shared", "-pthread",
+                           str(c_path), "-o", str(so_path)])
+    real = oracle._load()
+    lib = ctypes.CDLL(str(so_path))
+    lib.gdn_oracle_scan.argtypes = real.gdn_oracle_scan.argtypes
+    lib.gdn_oracle_scan.restype = ctypes.c_int
+    failed = []
+    oracle._lib = lib
+    try:
+        for name, fn in _pin_functions():
+            try:
+                fn()
+            except AssertionError:
+                failed.append(name)
+    finally:
+        oracle._lib = real
+    assert failed, "no pin caught the planted mistake %r" % mutation
