@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 gated delta-net scan (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+A step is one pass of the whole scan over one batch of synthetic inputs that
+are already resident in HBM: for the default workload, stream480
+(B=1, H=12, T=32,760, d_k=d_v=128, bf16 q/k/v, fp32 gates, fp32 output and
+state), one gdn_scan_causal call.  Its inputs (~500 MB) are larger than the
+126 MB L2, so no flush is needed between steps; for workloads smaller than
+L2 a 256 MB buffer is written between timed steps, outside the events.
+
+Metric: Mtokens/s = B*H*T per step / step time.  Time is measured with CUDA
+events on the launching stream after W warm-up steps, bracketed by a barrier
+and a device synchronise; with N > 1 (torchrun, one rank per GPU) every rank
+runs the same workload as an independent problem (weak scaling, no data-path
+collective) and the max over ranks is used.
+
+Extra keys: `roofline` (the dominant kernel's algorithmic bytes or FLOPs per
+launch over its mean CUDA-event duration in the same timed region, against
+the measured peak), `cpu_baseline` (the FP64 oracle on a bounded sample, on
+the host cores; rank 0 at N = 1), `e2e` (the same metric through the Python
+API with the inputs copied from pinned host memory and the output and state
+read back inside the timed region), `clocks` (nvidia-smi samples taken during
+the timed region) and `gpu_launches` (kernels the library launched in the
+timed region, from its own launch counter).
+
+`--impl reference` times the FP64 oracle (the reference implementation of
+this build) on the host cores instead: each step is a bounded sample of the
+same workload.
+"""
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "gated-delta scan Mtokens/s (B·H·T) on 1 B200; % of roofline"
+UNIT = "Mtokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+# Roofline denominators: measured on this machine's B200s (MEASURED_PEAKS.json)
+# when present, else the earlier pool measurement.
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic traffic and work (per token-head), see the design doc section 6
+# ---------------------------------------------------------------------------
+def bytes_per_token_head(w, out_bytes=4):
+    ib = 4 if w.dtype == "f32" else 2
+    return ib * (2 * w.dk + w.dv) + out_bytes * w.dv + 8   # q,k,v read; o written; alpha,beta
+
+
+def state_bytes_per_call(w):
+    return w.B * w.H * w.dk * w.dv * 4
+
+
+def flops_per_token_head(w, C=64):
+    dk, dv = w.dk, w.dv
+    causal = C * (6 * dk + 4 * dv) + 6 * dk * dv + C * C / 3.0
+    if w.mode == "bidir":
+        return causal + C * (2 * dk + 4 * dv) + 6 * dk * dv + C * C / 3.0
+    return causal
+
+
+def algorithmic_bytes_per_step(w):
+    b = w.token_heads * bytes_per_token_head(w)
+    if w.mode == "rollout":
+        b += w.calls * 2 * state_bytes_per_call(w)       # state read + written per call
+    elif w.mode == "causal":
+        b += state_bytes_per_call(w)                     # final state written
+    return b
+
+
+# Per kernel: which algorithmic bytes (per token-head) it moves.  The prep
+# kernel reads q, k, v and the gates; the chain kernel writes o (and the
+# state).  A fused kernel moves all of them.
+def kernel_algorithmic_bytes(name, w):
+    ib = 4 if w.dtype == "f32" else 2
+    reads = ib * (2 * w.dk + w.dv) + 8
+    writes = 4 * w.dv
+    if "prep" in name:
+        return reads
+    if "chain" in name:
+        return writes
+    return reads + writes
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_indices):
+        self.idx = set(gpu_indices)
+        self.proc = None
+        self.path = os.path.join("/tmp", "gdn_bench_clocks_%d.csv" % os.getpid())
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + SMI_FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    if int(parts[0]) not in self.idx:
+                        continue
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the workload's step on the GPU
+# ---------------------------------------------------------------------------
+class GPUStep:
+    def __init__(self, w, device):
+        import torch
+        import gated_delta_rule_72_b200 as gdn
+        from gated_delta_rule_72_b200 import inputs
+        self.torch, self.gdn, self.w, self.dev = torch, gdn, w, device
+        host = inputs.workload_inputs(w)          # drawn on the CPU, seeded
+        self.host = host
+        self.d = {n: t.to(device) for n, t in host.items()}
+        torch.cuda.synchronize(device)
+        self.o = torch.empty(w.B, w.total_T, w.H, w.dv, dtype=torch.float32, device=device)
+        self.state = torch.zeros(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)
+        td = self.d["q"].dtype
+        if w.mode == "rollout":
+            nb = gdn.workspace_size(w.B, w.T, w.H, w.dk, w.dv, td)
+            self.slices = []
+            for i in range(w.calls):
+                sl = slice(i * w.T, (i + 1) * w.T)
+                self.slices.append(({n: t[:, sl] for n, t in self.d.items()}, self.o[:, sl]))
+        else:
+            nb = gdn.workspace_size(w.B, w.T, w.H, w.dk, w.dv, td, bidir=(w.mode == "bidir"))
+        self.ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=device)
+        self.flush = None
+        in_bytes = sum(t.numel() * t.element_size() for t in self.d.values())
+        if in_bytes < 2 * L2_BYTES:
+            self.flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
+
+    def run(self):
+        gdn, d, w = self.gdn, self.d, self.w
+        if w.mode == "causal":
+            gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"], None, out=self.o,
+                            state_out=self.state, workspace=self.ws)
+        elif w.mode == "bidir":
+            gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"], out=self.o,
+                           workspace=self.ws)
+        else:
+            self.state.zero_()
+            for part, o in self.slices:
+                gdn.step(part["q"], part["k"], part["v"], part["alpha"], part["beta"], self.state,
+                         out=o, workspace=self.ws)
+
+    def between(self):
+        if self.flush is not None:
+            self.flush.fill_(1)
+
+    def run_e2e(self, pinned, dev_bufs, out_host, state_host):
+        """One end-to-end step through the public API: H2D of the inputs from
+        pinned memory, the scan, D2H of the output and the final state."""
+        for n, t in pinned.items():
+            dev_bufs[n].copy_(t, non_blocking=True)
+        gdn, d, w = self.gdn, dev_bufs, self.w
+        if w.mode == "causal":
+            gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"], None, out=self.o,
+                            state_out=self.state, workspace=self.ws)
+        elif w.mode == "bidir":
+            gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"], out=self.o,
+                           workspace=self.ws)
+        else:
+            self.state.zero_()
+            for i in range(w.calls):
+                sl = slice(i * w.T, (i + 1) * w.T)
+                gdn.step(d["q"][:, sl], d["k"][:, sl], d["v"][:, sl], d["alpha"][:, sl],
+                         d["beta"][:, sl], self.state, out=self.o[:, sl], workspace=self.ws)
+        out_host.copy_(self.o, non_blocking=True)
+        if state_host is not None:
+            state_host.copy_(self.state, non_blocking=True)
+
+
+def timed(torch, fn, between, steps, dist=None):
+    """Mean device ms per step over `steps` steps, CUDA events on the current stream."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s, e in ev:
+        between()
+        s.record()
+        fn()
+        e.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    return sum(s.elapsed_time(e) for s, e in ev) / steps
+
+
+def max_over_ranks(torch, dist, x, device):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# the FP64 oracle on the host cores (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_sample(w, target_s):
+    """Time the oracle on the first T_s tokens of every head, T_s sized so the
+    run takes about target_s seconds.  Returns (Mtok/s, threads, description)."""
+    import oracle
+    from gated_delta_rule_72_b200 import inputs
+    threads = max(1, min(os.cpu_count() or 1, w.B * w.H))
+    mode = "bidir" if w.mode == "bidir" else "causal"
+    full_T = w.total_T
+
+    def run(Ts):
+        x = inputs.generate(w.B, Ts, w.H, w.dk, w.dv, w.dtype, w.seed, w.gates)
+        t0 = time.perf_counter()
+        oracle.scan(x["q"], x["k"], x["v"], x["alpha"], x["beta"], mode=mode, threads=threads)
+        return time.perf_counter() - t0
+
+    Tc = min(full_T, 128)
+    tc = run(Tc)
+    Ts = int(min(full_T, max(Tc, Tc * target_s / max(tc, 1e-6))))
+    ts = run(Ts)
+    units = w.B * w.H * Ts
+    desc = "%s: all %d heads x first %d of %d tokens (%s), float64, %d threads" % (
+        w.name, w.B * w.H, Ts, full_T, mode, threads)
+    return units / ts / 1e6, threads, desc, Ts
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="stream480",
+                    choices=["stream480", "bidir720", "rollout", "skewed", "tiny"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target length of the oracle CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    from gated_delta_rule_72_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    config = {"workload": "%s (%s B=%d H=%d T=%d%s d_k=%d d_v=%d, %s in, fp32 out/state, %s gates)"
+              % (w.name, w.mode, w.B, w.H, w.T, (" x %d calls" % w.calls) if w.calls > 1 else "",
+                 w.dk, w.dv, w.dtype, w.gates),
+              "B": w.B, "H": w.H, "T": w.total_T, "d_k": w.dk, "d_v": w.dv, "chunk": 64,
+              "parallelism": "replicas%d (independent (b,h) problems per GPU)" % args.gpus}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        per_step_s = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+        import oracle  # noqa: F401  (the reference arm of this build is the oracle)
+        rate, threads, desc, Ts = oracle_sample(w, per_step_s)
+        # W warm-up + K timed steps, each the same bounded sample
+        from gated_delta_rule_72_b200 import inputs as I
+        x = I.generate(w.B, Ts, w.H, w.dk, w.dv, w.dtype, w.seed, w.gates)
+        mode = "bidir" if w.mode == "bidir" else "causal"
+        for _ in range(args.warmup):
+            oracle.scan(x["q"], x["k"], x["v"], x["alpha"], x["beta"], mode=mode, threads=threads)
+        times = []
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            oracle.scan(x["q"], x["k"], x["v"], x["alpha"], x["beta"], mode=mode, threads=threads)
+            times.append(time.perf_counter() - t0)
+        step_s = sum(times) / len(times)
+        value = w.B * w.H * Ts / step_s / 1e6
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": dict(config, sample_tokens_per_head=Ts),
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                 "sample": desc},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0},
+                "gpu_launches": 0}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import gated_delta_rule_72_b200 as gdn
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        torch.cuda.set_device(local)
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        dist = dist_mod
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    gdn.load()
+
+    step = GPUStep(w, device)
+    for _ in range(max(3, args.warmup)):
+        step.between()
+        step.run()
+    torch.cuda.synchronize()
+
+    # ---- the timed region: K steps, per-kernel events on, clocks sampled
+    sampler = ClockSampler(range(args.gpus)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+        for _ in range(2):       # keep the GPU busy while nvidia-smi starts
+            step.run()
+    gdn.gdn_read_kernel_timing()                  # drop anything recorded so far
+    n0 = gdn.gdn_launch_count()
+    gdn.gdn_set_kernel_timing(1)
+    ms = timed(torch, step.run, step.between, args.steps, dist)
+    gdn.gdn_set_kernel_timing(0)
+    launches = gdn.gdn_launch_count() - n0
+    clocks = sampler.stop() if sampler else None
+    ktimes = gdn.gdn_read_kernel_timing()
+    ms = max_over_ranks(torch, dist, ms, device)
+
+    units = w.token_heads                          # per GPU per step
+    value = args.gpus * units / (ms * 1e-3) / 1e6
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    dom = max(ktimes.items(), key=lambda kv: kv[1][0]) if ktimes else None
+    roof = None
+    if dom:
+        name, (tot_ms, n) = dom
+        per_launch_ms = tot_ms / n
+        launches_per_step = n / args.steps
+        units_per_launch = units / launches_per_step
+        bound = "tensor" if w.mode == "bidir" and "chain" not in name else "hbm"
+        if bound == "hbm":
+            alg = kernel_algorithmic_bytes(name, w) * units_per_launch
+            achieved = alg / (per_launch_ms * 1e-3) / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+        else:
+            alg = flops_per_token_head(w) * units_per_launch
+            achieved = alg / (per_launch_ms * 1e-3) / 1e12
+            peak = peaks["bf16_tflops"]
+            unit = "TFLOP/s"
+        total_ms = sum(t for t, _ in ktimes.values())
+        roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": None, "kernel": name,
+                "peak_source": "%s (%s)" % (peak_src, "MEASURED_PEAKS.json" if peak_src == "measured"
+                                            else "pool fallback"),
+                "kernel_ms_per_launch": per_launch_ms,
+                "kernel_share": tot_ms / total_ms if total_ms else None,
+                "kernels": {k: {"ms_per_step": t / args.steps, "launches_per_step": c / args.steps}
+                            for k, (t, c) in ktimes.items()}}
+    # whole step against its roofline (bytes at HBM bandwidth vs FLOPs at tensor peak)
+    t_mem = algorithmic_bytes_per_step(w) / (peaks["hbm_gbs"] * 1e9)
+    t_flop = w.token_heads * flops_per_token_head(w) / (peaks["bf16_tflops"] * 1e12)
+    step_roof = {"t_roofline_ms": max(t_mem, t_flop) * 1e3,
+                 "bound": "hbm" if t_mem >= t_flop else "tensor",
+                 "frac": max(t_mem, t_flop) / (ms * 1e-3)}
+
+    # ---- end to end through the public API, host buffers
+    pinned = {n: t.pin_memory() for n, t in step.host.items()}
+    dev_bufs = {n: torch.empty_like(t, device=device) for n, t in step.host.items()}
+    out_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
+    state_host = torch.empty(step.state.shape, dtype=torch.float32).pin_memory()
+    e2e_fn = lambda: step.run_e2e(pinned, dev_bufs, out_host, state_host)
+    for _ in range(2):
+        e2e_fn()
+    e2e_ms = timed(torch, e2e_fn, step.between, args.steps, dist)
+    e2e_ms = max_over_ranks(torch, dist, e2e_ms, device)
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = out_host.numel() * 4 + state_host.numel() * 4
+
+    # ---- oracle baseline on the host cores (rank 0, N = 1)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, threads, desc, _ = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": dict(config, l2=("inputs larger than L2, no flush" if step.flush is None
+                                           else "L2 flushed between steps (256 MB write)")),
+                "roofline": roof, "step_roofline": step_roof,
+                "cpu_baseline": cpu,
+                "e2e": {"value": args.gpus * units / (e2e_ms * 1e-3) / 1e6, "unit": UNIT,
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                        "ms_per_step": e2e_ms},
+                "clocks": clocks, "gpu_launches": launches}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,269 @@
+// gdn_api.cu -- the C-ABI entry points of libgdn.so: argument checks,
+// workspace planning and kernel dispatch.  See include/gdn.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/gdn.h"
+#include "common.cuh"
+#include "launch_stats.cuh"
+#include "simt_kernels.cuh"
+
+namespace {
+
+using gdn::kChunk;
+
+struct Args {
+    const void *q, *k, *v;
+    const float *alpha, *beta;
+    const float *state_in;
+    float *state_out;
+    void *o;
+    int B, T, H, dk, dv;
+    gdn_dtype dt, o_dt;
+    void *ws;
+    size_t ws_bytes;
+    cudaStream_t stream;
+};
+
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------
+// Workspace plan of the CUDA-core path: one fp32 record per chunk, head and
+// direction, then (bidirectional only) an fp32 partial output [B,T,H,dv].
+// ---------------------------------------------------------------------------
+size_t simt_record_floats(int dk, int dv) {
+    return (size_t)3 * kChunk * dk + (size_t)kChunk * dv + (size_t)kChunk * kChunk + 4;
+}
+
+size_t simt_workspace(int B, int T, int H, int dk, int dv, int bidir) {
+    const size_t nC = (size_t)(T + kChunk - 1) / kChunk;
+    const size_t ndir = bidir ? 2 : 1;
+    size_t bytes = round_up(ndir * B * H * nC * simt_record_floats(dk, dv) * sizeof(float), 256);
+    if (bidir) bytes += round_up((size_t)B * T * H * dv * sizeof(float), 256);
+    return bytes;
+}
+
+gdn_status check_common(const Args &a, bool need_inputs) {
+    if (a.dt != GDN_F32 && a.dt != GDN_BF16) return GDN_ERR_DTYPE;
+    if (a.o_dt != GDN_F32 && a.o_dt != GDN_BF16) return GDN_ERR_DTYPE;
+    if (a.B < 1 || a.H < 1 || a.T < 0) return GDN_ERR_SHAPE;
+    if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128))) return GDN_ERR_UNSUPPORTED;
+    // index arithmetic is 64-bit, but the chunk count and grid dims are int
+    if ((long long)a.B * a.H > 65535LL || a.T > (1 << 30)) return GDN_ERR_SHAPE;
+    if (need_inputs) {
+        if (!a.q || !a.k || !a.v || !a.alpha || !a.beta || !a.o) return GDN_ERR_NULL;
+        const void *ps[] = {a.q, a.k, a.v, a.o};
+        for (const void *p : ps)
+            if (!aligned(p, 16)) return GDN_ERR_ALIGN;
+        // the gates are read one float at a time
+        if (!aligned(a.alpha, 4) || !aligned(a.beta, 4)) return GDN_ERR_ALIGN;
+    }
+    if (a.state_in && !aligned(a.state_in, 16)) return GDN_ERR_ALIGN;
+    if (a.state_out && !aligned(a.state_out, 16)) return GDN_ERR_ALIGN;
+    if (a.state_in && a.state_out && a.state_in != a.state_out) {
+        const size_t n = (size_t)a.B * a.H * a.dk * a.dv * sizeof(float);
+        const char *i0 = (const char *)a.state_in, *o0 = (const char *)a.state_out;
+        if (i0 < o0 + n && o0 < i0 + n) return GDN_ERR_SHAPE;  // partial overlap
+    }
+    return GDN_OK;
+}
+
+gdn_status check_ws(const Args &a, size_t need) {
+    if (need == 0) return GDN_OK;
+    if (!a.ws) return GDN_ERR_NULL;
+    if (!aligned(a.ws, 256)) return GDN_ERR_ALIGN;
+    if (a.ws_bytes < need) return GDN_ERR_WORKSPACE;
+    return GDN_OK;
+}
+
+gdn_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// T = 0: state_out <- state_in (or zero).
+gdn_status empty_scan(const Args &a) {
+    if (!a.state_out || a.state_out == a.state_in) return GDN_OK;
+    const size_t n = (size_t)a.B * a.H * a.dk * a.dv * sizeof(float);
+    cudaError_t e = a.state_in
+        ? cudaMemcpyAsync(a.state_out, a.state_in, n, cudaMemcpyDeviceToDevice, a.stream)
+        : cudaMemsetAsync(a.state_out, 0, n, a.stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core path
+// ---------------------------------------------------------------------------
+template <int DK, int DV, typename Tin, typename Tout>
+gdn_status run_simt(const Args &a, int bidir) {
+    using namespace gdn::simt;
+    constexpr int NS = 32;
+    const int nC = (a.T + kChunk - 1) / kChunk;
+    const int nbh = a.B * a.H;
+    float *rec = static_cast<float *>(a.ws);
+    const size_t rec_bytes = round_up((size_t)(bidir ? 2 : 1) * nbh * nC *
+                                      Record<DK, DV>::kFloats * sizeof(float), 256);
+    float *part = bidir ? reinterpret_cast<float *>(static_cast<char *>(a.ws) + rec_bytes) : nullptr;
+
+    auto prep = prep_kernel<DK, DV, Tin>;
+    const size_t prep_smem = PrepSmem<DK, DV>::kBytes;
+    if (cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    {
+        gdn::LaunchScope ls("simt_prep", a.stream);
+        prep<<<dim3(nC, nbh, bidir ? 2 : 1), 256, prep_smem, a.stream>>>(
+            static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
+            static_cast<const Tin *>(a.v), a.alpha, a.beta, rec, a.T, a.H, nC, 0);
+    }
+    if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
+
+    auto chain = chain_kernel<DK, DV, NS, Tout>;
+    const size_t chain_smem = ChainSmem<DK, NS>::kBytes;
+    if (cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chain_smem) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const dim3 grid(DV / NS, nbh, 1);
+    Tout *o = static_cast<Tout *>(a.o);
+    if (!bidir) {
+        gdn::LaunchScope ls("simt_chain", a.stream);
+        chain<<<grid, 256, chain_smem, a.stream>>>(rec, a.state_in, a.state_out, o, nullptr,
+                                                   a.T, a.H, nC, 0, kOutStore, nbh);
+        return launch_status();
+    }
+    {
+        gdn::LaunchScope ls("simt_chain", a.stream);
+        chain<<<grid, 256, chain_smem, a.stream>>>(rec, nullptr, nullptr, o, part, a.T, a.H, nC,
+                                                   0, kOutPartial, nbh);
+    }
+    if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
+    gdn::LaunchScope ls("simt_chain", a.stream);
+    chain<<<grid, 256, chain_smem, a.stream>>>(rec, nullptr, nullptr, o, part, a.T, a.H, nC, 1,
+                                               kOutAddPartial, nbh);
+    return launch_status();
+}
+
+template <typename Tin, typename Tout>
+gdn_status dispatch_dims(const Args &a, int bidir) {
+    if (a.dk == 128 && a.dv == 128) return run_simt<128, 128, Tin, Tout>(a, bidir);
+    if (a.dk == 128 && a.dv == 64) return run_simt<128, 64, Tin, Tout>(a, bidir);
+    if (a.dk == 64 && a.dv == 128) return run_simt<64, 128, Tin, Tout>(a, bidir);
+    return run_simt<64, 64, Tin, Tout>(a, bidir);
+}
+
+template <typename Tin>
+gdn_status dispatch_out(const Args &a, int bidir) {
+    return a.o_dt == GDN_F32 ? dispatch_dims<Tin, float>(a, bidir)
+                             : dispatch_dims<Tin, __nv_bfloat16>(a, bidir);
+}
+
+size_t plan_workspace(int B, int T, int H, int dk, int dv, int bidir) {
+    if (T == 0) return 0;
+    return simt_workspace(B, T, H, dk, dv, bidir);
+}
+
+gdn_status run(const Args &a, int bidir) {
+    const gdn_status s = check_ws(a, plan_workspace(a.B, a.T, a.H, a.dk, a.dv, bidir));
+    if (s != GDN_OK) return s;
+    if (a.T == 0) return bidir ? GDN_OK : empty_scan(a);
+    return a.dt == GDN_F32 ? dispatch_out<float>(a, bidir) : dispatch_out<__nv_bfloat16>(a, bidir);
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_scan_causal(const void *q, const void *k, const void *v, const float *alpha,
+                           const float *beta, const float *state_in, float *state_out, void *o,
+                           int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt,
+                           void *workspace, size_t ws_bytes, void *stream) {
+    Args a{q, k, v, alpha, beta, state_in, state_out, o, B, T, H, dk, dv, dt, o_dt,
+           workspace, ws_bytes, static_cast<cudaStream_t>(stream)};
+    gdn_status s = check_common(a, T > 0);
+    if (s != GDN_OK) return s;
+    return run(a, 0);
+}
+
+gdn_status gdn_scan_bidir(const void *q, const void *k, const void *v, const float *alpha,
+                          const float *beta, void *o, int B, int T, int H, int dk, int dv,
+                          gdn_dtype dt, gdn_dtype o_dt, void *workspace, size_t ws_bytes,
+                          void *stream) {
+    Args a{q, k, v, alpha, beta, nullptr, nullptr, o, B, T, H, dk, dv, dt, o_dt,
+           workspace, ws_bytes, static_cast<cudaStream_t>(stream)};
+    gdn_status s = check_common(a, T > 0);
+    if (s != GDN_OK) return s;
+    return run(a, 1);
+}
+
+gdn_status gdn_step(const void *q, const void *k, const void *v, const float *alpha,
+                    const float *beta, float *state, void *o, int B, int T, int H, int dk, int dv,
+                    gdn_dtype dt, gdn_dtype o_dt, void *workspace, size_t ws_bytes, void *stream) {
+    if (!state) return GDN_ERR_NULL;
+    Args a{q, k, v, alpha, beta, state, state, o, B, T, H, dk, dv, dt, o_dt,
+           workspace, ws_bytes, static_cast<cudaStream_t>(stream)};
+    gdn_status s = check_common(a, T > 0);
+    if (s != GDN_OK) return s;
+    return run(a, 0);
+}
+
+size_t gdn_workspace_size(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt,
+                          int bidir) {
+    Args a{};
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.dt = dt; a.o_dt = o_dt;
+    if (check_common(a, false) != GDN_OK) return 0;
+    return plan_workspace(B, T, H, dk, dv, bidir ? 1 : 0);
+}
+
+const char *gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_NULL: return "a required pointer is NULL";
+        case GDN_ERR_SHAPE: return "bad shape (B<1, H<1, T<0, size overflow, or overlapping state buffers)";
+        case GDN_ERR_DTYPE: return "unknown dtype";
+        case GDN_ERR_ALIGN: return "pointer not 16-byte aligned (workspace: 256-byte)";
+        case GDN_ERR_UNSUPPORTED: return "unsupported head dimension (dk, dv must be 64 or 128)";
+        case GDN_ERR_WORKSPACE: return "workspace smaller than gdn_workspace_size()";
+        case GDN_ERR_CUDA: return "CUDA launch or copy failed";
+    }
+    return "unknown status";
+}
+
+const char *gdn_version(void) { return "gdn-b200 0.1 (sm_100a)"; }
+
+unsigned long long gdn_launch_count(void) {
+    return gdn::LaunchStats::get().launches.load(std::memory_order_relaxed);
+}
+
+void gdn_set_kernel_timing(int on) { gdn::LaunchStats::get().timing.store(on != 0); }
+
+int gdn_read_kernel_timing(char *names, int name_len, double *total_ms, int *launches, int max) {
+    if (max < 0 || name_len < 1) return GDN_ERR_SHAPE;
+    if (max > 0 && (!names || !total_ms || !launches)) return GDN_ERR_NULL;
+    gdn::LaunchStats &st = gdn::LaunchStats::get();
+    std::lock_guard<std::mutex> g(st.mu);
+    int n = 0;
+    gdn_status status = GDN_OK;
+    for (auto &e : st.events) {
+        double ms = 0.0;
+        for (auto &pr : e.second) {
+            float t = 0.f;
+            if (cudaEventSynchronize(pr.second) != cudaSuccess ||
+                cudaEventElapsedTime(&t, pr.first, pr.second) != cudaSuccess)
+                status = GDN_ERR_CUDA;
+            ms += t;
+            cudaEventDestroy(pr.first);
+            cudaEventDestroy(pr.second);
+        }
+        if (n < max) {
+            strncpy(names + (size_t)n * name_len, e.first.c_str(), name_len - 1);
+            names[(size_t)n * name_len + name_len - 1] = 0;
+            total_ms[n] = ms;
+            launches[n] = (int)e.second.size();
+            ++n;
+        }
+    }
+    st.events.clear();
+    return status == GDN_OK ? n : status;
+}
+
+}  // extern "C"

@@ -1,0 +1,155 @@
+/*
+ * gdn.h -- C-ABI of the B200 (sm_100a) gated delta-net scan library, libgdn.so.
+ *
+ * The operator (per batch b and head h, t = 1..T, state S of d_k x d_v with
+ * the key dimension as the row index):
+ *
+ *     S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * This is gated delta-net linear attention with a matrix-valued recurrent
+ * state per head.  The issue "[Research] Explore linear attention for the
+ * streaming video models" (sections "We already ship a hybrid
+ * linear-attention model" and "Open questions and risks") asks for its
+ * causal, forward-only form with the state carried across calls.  The
+ * bidirectional form follows "Video DeltaNet" (AI summary, "Methodology in
+ * Plain English"): a forward and a backward state cover disjoint regions
+ * and their readouts are added.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  Layout   q, k : [B, T, H, dk]   v : [B, T, H, dv]   element type `dt`
+ *           o : [B, T, H, dv] element type `o_dt` (GDN_F32 or GDN_BF16)
+ *           all contiguous, row-major
+ *           alpha, beta : [B, T, H] fp32;  alpha in (0, 1], beta in [0, 1]
+ *           state : [B, H, dk, dv] fp32, row index = key dimension
+ *  Sizes    B >= 1, H >= 1, T >= 0; dk, dv in {64, 128}.
+ *  Pointers All tensor pointers are DEVICE pointers, 16-byte aligned (alpha
+ *           and beta: 4-byte aligned, so a token slice of them is valid).  The
+ *           caller owns every buffer, including the workspace; the library
+ *           never allocates, frees or synchronises.  Every call is
+ *           asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *           stream) and performs no host synchronisation, so a call can be
+ *           captured in a CUDA graph.
+ *  Workspace `workspace` must hold at least gdn_workspace_size(...) bytes
+ *           for the same arguments, 256-byte aligned; it may be NULL when
+ *           that size is 0.  Its contents on entry do not matter.
+ *  Errors   Arguments are checked on the host before any launch; a bad
+ *           argument returns a negative gdn_status and launches nothing.
+ *           A failed launch returns GDN_ERR_CUDA.  Kernels never trap.
+ *  Inputs   alpha must be > 0 (the kernels use log alpha); values outside
+ *           the stated ranges are not detected and give unspecified
+ *           results, but never out-of-bounds accesses.
+ *  Output   State and accumulation are fp32 whatever `dt` is.  With
+ *           o_dt = GDN_F32 the output is the fp32 accumulator; with
+ *           GDN_BF16 it is rounded once to bf16 (round to nearest even).
+ *           Rounding to bf16 alone moves max|o|/rms(o) by up to 2^-8 times
+ *           max|o|/rms(o), which on long sequences is several 1e-2, so the
+ *           fp32 output is the one that carries the accuracy of the scan.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_NULL = -1,        /* a required pointer is NULL */
+    GDN_ERR_SHAPE = -2,       /* B < 1, H < 1, T < 0, or a size overflows */
+    GDN_ERR_DTYPE = -3,       /* dt or o_dt is not a gdn_dtype */
+    GDN_ERR_ALIGN = -4,       /* a pointer is not 16-byte (workspace: 256-byte) aligned */
+    GDN_ERR_UNSUPPORTED = -5, /* dk or dv not in {64, 128} */
+    GDN_ERR_WORKSPACE = -6,   /* ws_bytes < gdn_workspace_size(...) */
+    GDN_ERR_CUDA = -7         /* a CUDA launch or copy failed */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/*
+ * gdn_scan_causal -- causal scan over T tokens with optional state in/out.
+ *   state_in   initial state S_0, or NULL for zero.
+ *   state_out  receives S_T, or NULL (not written).  May equal state_in
+ *              (in-place update); must not overlap it otherwise.
+ *   o          receives o_1..o_T.
+ * T = 0 writes state_out <- state_in (zero if state_in is NULL) and no o.
+ */
+GDN_API gdn_status gdn_scan_causal(const void *q, const void *k, const void *v,
+                           const float *alpha, const float *beta,
+                           const float *state_in, float *state_out, void *o,
+                           int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * gdn_scan_bidir -- bidirectional scan:
+ *     o_t = S_t^T q_t + R_{t+1}^T q_t,
+ *     R_t = alpha_t (I - beta_t k_t k_t^T) R_{t+1} + beta_t k_t v_t^T,  R_{T+1} = 0,
+ * i.e. the causal scan from zero plus the same recurrence run from T down
+ * to 1, read before token t is written (token t is counted once, by the
+ * causal part).  The two readouts are summed in fp32 (and, for a bf16
+ * output, rounded once).
+ */
+GDN_API gdn_status gdn_scan_bidir(const void *q, const void *k, const void *v,
+                          const float *alpha, const float *beta, void *o,
+                          int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt,
+                          void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * gdn_step -- one streaming call: gdn_scan_causal with state_in == state_out
+ * == state (required, updated in place).  A rollout is a sequence of
+ * gdn_step calls on successive slices of the token stream; the result equals
+ * one gdn_scan_causal over the concatenated tokens up to rounding.
+ */
+GDN_API gdn_status gdn_step(const void *q, const void *k, const void *v,
+                    const float *alpha, const float *beta, float *state, void *o,
+                    int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt,
+                    void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * gdn_workspace_size -- bytes of device workspace a call with these
+ * arguments needs (bidir != 0: gdn_scan_bidir; else gdn_scan_causal /
+ * gdn_step).  Returns 0 for arguments that the call would reject.
+ */
+GDN_API size_t gdn_workspace_size(int B, int T, int H, int dk, int dv, gdn_dtype dt,
+                                  gdn_dtype o_dt, int bidir);
+
+/* gdn_status_string -- static, NUL-terminated description of a status. */
+GDN_API const char *gdn_status_string(gdn_status s);
+
+/* gdn_version -- static version string of the library build. */
+GDN_API const char *gdn_version(void);
+
+/*
+ * Introspection (measurement support; not part of the scan itself).
+ *
+ * gdn_launch_count -- number of CUDA kernels this library has launched in
+ *   this process so far (all devices, all threads).
+ * gdn_set_kernel_timing -- on != 0: from now on, bracket every kernel launch
+ *   with a pair of CUDA events recorded on the launch stream; 0: stop.  Use
+ *   only on eager (not graph-captured) calls.  Creating the events is the
+ *   only host-side work it adds; it never synchronises.
+ * gdn_read_kernel_timing -- synchronise on the recorded events, then report
+ *   per kernel name (at most `max` names): total device milliseconds and the
+ *   number of launches since the previous read, and forget them.  `names`
+ *   receives `max` NUL-terminated slots of `name_len` bytes.  Returns the
+ *   number of kernel names written, or a negative gdn_status.
+ */
+GDN_API unsigned long long gdn_launch_count(void);
+GDN_API void gdn_set_kernel_timing(int on);
+GDN_API int gdn_read_kernel_timing(char *names, int name_len, double *total_ms, int *launches,
+                                   int max);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -1,0 +1,129 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+that include/gdn.h declares, and rejects bad arguments on the host before
+any CUDA call (fake pointers are never dereferenced on these paths)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_72_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for required in ("gdn_scan_causal", "gdn_scan_bidir", "gdn_step", "gdn_workspace_size",
+                     "gdn_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) <= set(_lib.SIGNATURES)
+
+
+def test_exports_nothing_undeclared():
+    out = os.popen("nm -D --defined-only %s" % _lib.LIB_PATH).read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert exported == set(_declared())
+
+
+def test_status_strings(lib):
+    for code in _lib.STATUS:
+        s = _lib.gdn_status_string(code)
+        assert s and s != "unknown status"
+    assert _lib.gdn_status_string(12345) == "unknown status"
+    assert "sm_100a" in _lib.gdn_version()
+
+
+def test_workspace_size_rules(lib):
+    assert _lib.gdn_workspace_size(1, 0, 2, 64, 64, 0, 0, 0) == 0          # T = 0: nothing
+    assert _lib.gdn_workspace_size(1, 256, 2, 96, 64, 0, 0, 0) == 0        # unsupported dk
+    assert _lib.gdn_workspace_size(0, 256, 2, 64, 64, 0, 0, 0) == 0        # B < 1
+    assert _lib.gdn_workspace_size(1, 256, 2, 64, 64, 7, 0, 0) == 0        # bad dtype
+    assert _lib.gdn_workspace_size(1, 256, 2, 64, 64, 0, 9, 0) == 0        # bad output dtype
+    a = _lib.gdn_workspace_size(1, 256, 2, 64, 64, 0, 0, 0)
+    b = _lib.gdn_workspace_size(1, 256, 2, 64, 64, 0, 0, 1)
+    assert a > 0 and b > a and a % 256 == 0 and b % 256 == 0
+    big = _lib.gdn_workspace_size(1, 75600, 20, 128, 128, 1, 0, 1)
+    assert big > 0
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced on the rejected paths
+
+
+def _causal(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, alpha=FAKE, beta=FAKE, state_in=None, state_out=None,
+                o=FAKE, B=1, T=64, H=2, dk=64, dv=64, dt=0, o_dt=0, workspace=FAKE, ws_bytes=1 << 40,
+                stream=None)
+    args.update(kw)
+    return _lib.gdn_scan_causal(*args.values())
+
+
+def test_rejects_before_launch(lib):
+    assert _causal(q=None) == -1
+    assert _causal(o=None) == -1
+    assert _causal(B=0) == -2
+    assert _causal(H=0) == -2
+    assert _causal(T=-1) == -2
+    assert _causal(dt=5) == -3
+    assert _causal(o_dt=-1) == -3
+    assert _causal(k=FAKE + 4) == -4
+    assert _causal(o=FAKE + 8) == -4
+    assert _causal(alpha=FAKE + 2) == -4
+    assert _causal(alpha=FAKE + 4, beta=FAKE + 8, ws_bytes=100) == -6  # gates need 4 bytes only
+    assert _causal(state_in=FAKE + 2) == -4
+    assert _causal(dk=96) == -5
+    assert _causal(dv=32) == -5
+    assert _causal(workspace=None) == -1
+    assert _causal(workspace=FAKE + 16) == -4        # workspace needs 256-byte alignment
+    assert _causal(ws_bytes=100) == -6
+    # state_in and state_out that overlap without being equal
+    assert _causal(state_in=FAKE, state_out=FAKE + 256) == -2
+
+
+def test_step_requires_state(lib):
+    st = _lib.gdn_step(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1, 64, 2, 64, 64, 0, 0, FAKE,
+                       1 << 40, None)
+    assert st == -1
+
+
+def test_bidir_rejects(lib):
+    st = _lib.gdn_scan_bidir(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, 2, 64, 128, 1, 0, FAKE, 10,
+                             None)
+    assert st == -6
+    st = _lib.gdn_scan_bidir(FAKE, None, FAKE, FAKE, FAKE, FAKE, 1, 64, 2, 64, 128, 1, 0, FAKE,
+                             1 << 40, None)
+    assert st == -1
+
+
+def test_empty_scan_without_state_is_a_noop(lib):
+    # T = 0, no state buffers: nothing to do, no CUDA call is made
+    assert _causal(T=0, q=None, k=None, v=None, alpha=None, beta=None, o=None, workspace=None,
+                   ws_bytes=0) == 0
+
+
+def test_python_api_refuses_cpu_tensors():
+    import torch
+    import gated_delta_rule_72_b200 as g
+    x = torch.zeros(1, 8, 1, 64)
+    a = torch.ones(1, 8, 1)
+    with pytest.raises(ValueError, match="CUDA"):
+        g.scan_causal(x, x, x, a, a)
+    with pytest.raises(ValueError, match="CUDA"):
+        g.scan_bidir(x, x, x, a, a)

@@ -1,0 +1,169 @@
+"""GPU parity: the CUDA library against the FP64 oracle, element by element,
+on the same seeded inputs.  Tolerance (max|gpu - oracle| / rms(oracle)):
+1e-4 for fp32 inputs, 2e-2 for bf16 inputs; the final state is held to the
+same bar against rms of the oracle's state."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_72_b200 as gdn
+from gated_delta_rule_72_b200 import inputs
+from tests.gpu_util import TOL, oracle_heads, rel_err, rel_err_bf16_out, to_dev
+
+pytestmark = pytest.mark.gpu
+
+DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def _state(B, H, dk, dv, seed):
+    g = torch.Generator("cpu").manual_seed(seed)
+    return (0.3 * torch.randn(B, H, dk, dv, generator=g)).float()
+
+
+def test_tiny_workload():
+    """B=1, H=2, T=256, d=64, fp32, chunk 64, seed 0."""
+    w = inputs.WORKLOADS["tiny"]
+    inp = inputs.workload_inputs(w)
+    d = to_dev(inp)
+    o, s = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle_heads(inp)
+    assert rel_err(o, o_ref) <= 1e-4
+    assert rel_err(s, s_ref) <= 1e-4
+
+
+SHAPES = [(64, 64), (128, 128), (64, 128), (128, 64)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", SHAPES)
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 200])
+def test_causal_shapes(dtype, dk, dv, T):
+    B, H = 2, 3
+    inp = inputs.generate(B, T, H, dk, dv, dtype, seed=1000 + T + dk + dv)
+    s0 = _state(B, H, dk, dv, seed=T)
+    d = to_dev(inp)
+    o, s = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"], s0.cuda())
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle_heads(inp, state_in=s0)
+    tol = TOL[DT[dtype]]
+    assert rel_err(o, o_ref) <= tol
+    assert rel_err(s, s_ref) <= tol
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (128, 64)])
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 130, 257])
+def test_bidir_shapes(dtype, dk, dv, T):
+    B, H = 1, 3
+    inp = inputs.generate(B, T, H, dk, dv, dtype, seed=2000 + T + dk)
+    d = to_dev(inp)
+    o = gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+    torch.cuda.synchronize()
+    o_ref, _ = oracle_heads(inp, mode="bidir")
+    assert rel_err(o, o_ref) <= TOL[DT[dtype]]
+
+
+@pytest.mark.parametrize("gates", ["default", "skewed"])
+def test_streaming_splits_match_one_call(gates):
+    """gdn_step over arbitrary call boundaries (lengths 1, 63, 64, 65, ...)
+    equals one causal scan, and both equal the oracle."""
+    B, T, H, dk, dv = 1, 600, 2, 128, 128
+    inp = inputs.generate(B, T, H, dk, dv, "bf16", seed=77, gates=gates)
+    d = to_dev(inp)
+    o_one, s_one = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+    cuts = [0, 1, 64, 127, 191, 192, 257, 300, 365, 429, 430, 599, 600]
+    state = torch.zeros(B, H, dk, dv, device="cuda")
+    outs = []
+    for a, b in zip(cuts, cuts[1:]):
+        sl = {n: t[:, a:b].contiguous() for n, t in d.items()}
+        outs.append(gdn.step(sl["q"], sl["k"], sl["v"], sl["alpha"], sl["beta"], state))
+    o_split = torch.cat(outs, dim=1)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle_heads(inp)
+    tol = TOL[torch.bfloat16]
+    assert rel_err(o_split, o_ref) <= tol
+    assert rel_err(state, s_ref) <= tol
+    assert rel_err(o_one, o_ref) <= tol
+    # the two GPU evaluations differ only by chunk boundaries
+    assert rel_err(o_split.float(), o_one.float().cpu().double().numpy()) <= tol
+
+
+def test_identity_gates_keep_state():
+    """alpha = 1, beta = 0: every token is an identity step, o_t = S_0^T q_t."""
+    B, T, H, dk, dv = 1, 100, 2, 64, 64
+    inp = inputs.generate(B, T, H, dk, dv, "f32", seed=5)
+    inp["alpha"] = torch.ones_like(inp["alpha"])
+    inp["beta"] = torch.zeros_like(inp["beta"])
+    s0 = _state(B, H, dk, dv, 9)
+    d = to_dev(inp)
+    o, s = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"], s0.cuda())
+    torch.cuda.synchronize()
+    want = torch.einsum("bthi,bhij->bthj", inp["q"].double(), s0.double())
+    assert rel_err(o, want.numpy()) <= 1e-5
+    assert torch.equal(s.cpu(), s0)
+
+
+def test_empty_sequence_passes_state():
+    B, H, dk, dv = 2, 3, 128, 64
+    s0 = _state(B, H, dk, dv, 3).cuda()
+    e = torch.empty(B, 0, H, dk, device="cuda")
+    ev = torch.empty(B, 0, H, dv, device="cuda")
+    g = torch.empty(B, 0, H, device="cuda")
+    o, s = gdn.scan_causal(e, e, ev, g, g, s0)
+    torch.cuda.synchronize()
+    assert o.shape == (B, 0, H, dv)
+    assert torch.equal(s, s0)
+    o, s = gdn.scan_causal(e, e, ev, g, g, None)
+    assert torch.count_nonzero(s) == 0
+    o = gdn.scan_bidir(e, e, ev, g, g)
+    assert o.shape == (B, 0, H, dv)
+
+
+def test_in_place_state_update():
+    B, T, H, dk, dv = 1, 130, 2, 64, 128
+    inp = inputs.generate(B, T, H, dk, dv, "f32", seed=11)
+    s0 = _state(B, H, dk, dv, 4)
+    d = to_dev(inp)
+    st = s0.cuda().clone()
+    o = gdn.step(d["q"], d["k"], d["v"], d["alpha"], d["beta"], st)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle_heads(inp, state_in=s0)
+    assert rel_err(o, o_ref) <= 1e-4
+    assert rel_err(st, s_ref) <= 1e-4
+
+
+@pytest.mark.parametrize("mode", ["causal", "bidir"])
+def test_bf16_output(mode):
+    """o_dt = bf16: the fp32 result rounded once; held to the bf16 bar after
+    allowing the rounding of the output itself (2^-8 relative per element)."""
+    B, T, H, dk, dv = 1, 333, 2, 128, 128
+    inp = inputs.generate(B, T, H, dk, dv, "bf16", seed=31)
+    d = to_dev(inp)
+    if mode == "causal":
+        o, _ = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
+                               out_dtype=torch.bfloat16)
+        o32, _ = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+    else:
+        o = gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"], out_dtype=torch.bfloat16)
+        o32 = gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+    torch.cuda.synchronize()
+    assert o.dtype == torch.bfloat16
+    o_ref, _ = oracle_heads(inp, mode=mode)
+    assert rel_err_bf16_out(o, o_ref) <= 2e-2
+    # the bf16 output is the fp32 output rounded once (round to nearest even)
+    assert torch.equal(o, o32.to(torch.bfloat16))
+
+
+def test_workspace_is_reusable_and_contents_do_not_matter():
+    B, T, H, dk, dv = 1, 200, 2, 128, 128
+    inp = inputs.generate(B, T, H, dk, dv, "bf16", seed=12)
+    d = to_dev(inp)
+    nb = gdn.workspace_size(B, T, H, dk, dv, torch.bfloat16, bidir=True)
+    ws = torch.full((nb,), 0x7F, dtype=torch.uint8, device="cuda")  # garbage (NaN-ish floats)
+    o1 = gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"], workspace=ws)
+    o2 = gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"], workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    o_ref, _ = oracle_heads(inp, mode="bidir")
+    assert rel_err(o1, o_ref) <= 2e-2
