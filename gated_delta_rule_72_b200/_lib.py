@@ -24,6 +24,7 @@ SIGNATURES = {
     "gdn_scan_causal": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "gdn_scan_bidir": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "gdn_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
+    "gdn_step_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "gdn_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gdn_status_string": (ctypes.c_char_p, [_I]),
     "gdn_version": (ctypes.c_char_p, []),
@@ -75,6 +76,14 @@ def gdn_step(q, k, v, alpha, beta, state, o, B, T, H, dk, dv, dt, o_dt, workspac
              stream):
     return load().gdn_step(q, k, v, alpha, beta, state, o, B, T, H, dk, dv, dt, o_dt, workspace,
                            ws_bytes, stream)
+
+
+def gdn_step_noalloc(q, k, v, alpha, beta, state, o, B, T, H, dk, dv, dt, o_dt, stream):
+    return load().gdn_step_noalloc(q, k, v, alpha, beta, state, o, B, T, H, dk, dv, dt, o_dt,
+                                   stream)
+
+
+GDN_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 def gdn_workspace_size(B, T, H, dk, dv, dt, o_dt, bidir):

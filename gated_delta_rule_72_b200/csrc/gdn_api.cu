@@ -4,6 +4,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/gdn.h"
 #include "common.cuh"
 #include "launch_stats.cuh"
@@ -171,6 +173,38 @@ gdn_status run(const Args &a, int bidir) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Scratch of gdn_step_noalloc: a file-scope device array, so that callers
+// who cannot allocate device memory still get the workspace a call needs.
+// Host code must not pass `g_noalloc_scratch` itself to a kernel (in host
+// code the name is a host-side stand-in, not a device address); the device
+// address is looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set up on the
+// first call per device, with that device current).
+gdn_status noalloc_scratch(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDN_ERR_CUDA;
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDN_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return GDN_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 gdn_status gdn_scan_causal(const void *q, const void *k, const void *v, const float *alpha,
@@ -203,6 +237,24 @@ gdn_status gdn_step(const void *q, const void *k, const void *v, const float *al
            workspace, ws_bytes, static_cast<cudaStream_t>(stream)};
     gdn_status s = check_common(a, T > 0);
     if (s != GDN_OK) return s;
+    return run(a, 0);
+}
+
+gdn_status gdn_step_noalloc(const void *q, const void *k, const void *v, const float *alpha,
+                            const float *beta, float *state, void *o, int B, int T, int H, int dk,
+                            int dv, gdn_dtype dt, gdn_dtype o_dt, void *stream) {
+    if (!state) return GDN_ERR_NULL;
+    Args a{q, k, v, alpha, beta, state, state, o, B, T, H, dk, dv, dt, o_dt,
+           nullptr, 0, static_cast<cudaStream_t>(stream)};
+    gdn_status s = check_common(a, T > 0);
+    if (s != GDN_OK) return s;
+    const size_t need = plan_workspace(B, T, H, dk, dv, 0);
+    if (need > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
+    if (need > 0) {
+        s = noalloc_scratch(&a.ws);
+        if (s != GDN_OK) return s;
+        a.ws_bytes = GDN_NOALLOC_SCRATCH_BYTES;
+    }
     return run(a, 0);
 }
 

@@ -115,6 +115,38 @@ GDN_API gdn_status gdn_step(const void *q, const void *k, const void *v,
                     void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * gdn_step_noalloc -- gdn_step for callers that cannot allocate device
+ * memory.  Some callers may not call cudaMalloc at all: code running inside
+ * a host framework that owns every byte of device memory through its own
+ * pool, or a real-time rollout loop where an allocation (which can
+ * synchronise the device) would stall the pipeline.  This entry point takes
+ * no workspace: its scratch is a file-scope __device__ array of
+ * GDN_NOALLOC_SCRATCH_BYTES (64 MiB) inside libgdn.so, which every GPU that
+ * loads the library holds until the process exits.  The caller still owns
+ * q, k, v, alpha, beta, state and o.  (The pages have no counterpart of
+ * this call; it exists for deployment only.)
+ *   - It runs on the current device.  Its first call on a device looks up the
+ *     array's device address (cudaGetSymbolAddress) with that device current;
+ *     make that first call before any stream capture.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Arguments whose gdn_workspace_size(..., bidir = 0) exceeds
+ *     GDN_NOALLOC_SCRATCH_BYTES are rejected with GDN_ERR_WORKSPACE before
+ *     any launch (for d = 128 and bf16 inputs that is roughly B*H*ceil(T/64)
+ *     > 450 chunk-heads).
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     nothing in it needs to start at zero (every scratch byte a call reads
+ *     was written earlier by the same call, in stream order).  Calls that
+ *     overlap on the GPU (different streams, or several host threads) race
+ *     on the array and give wrong results: serialise them.
+ * Semantics, layout and status codes are otherwise those of gdn_step.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+GDN_API gdn_status gdn_step_noalloc(const void *q, const void *k, const void *v,
+                                    const float *alpha, const float *beta, float *state, void *o,
+                                    int B, int T, int H, int dk, int dv, gdn_dtype dt,
+                                    gdn_dtype o_dt, void *stream);
+
+/*
  * gdn_workspace_size -- bytes of device workspace a call with these
  * arguments needs (bidir != 0: gdn_scan_bidir; else gdn_scan_causal /
  * gdn_step).  Returns 0 for arguments that the call would reject.

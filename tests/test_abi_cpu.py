@@ -127,3 +127,16 @@ def test_python_api_refuses_cpu_tensors():
         g.scan_causal(x, x, x, a, a)
     with pytest.raises(ValueError, match="CUDA"):
         g.scan_bidir(x, x, x, a, a)
+
+
+def test_noalloc_rejects_oversized_before_launch(lib):
+    """gdn_step_noalloc refuses work whose scratch would exceed its fixed
+    array, before touching the GPU (fake pointers are never used)."""
+    B, T, H, d = 1, 64 * 2000, 16, 128
+    assert _lib.gdn_workspace_size(B, T, H, d, d, 1, 0, 0) > _lib.GDN_NOALLOC_SCRATCH_BYTES
+    st = _lib.gdn_step_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, B, T, H, d, d, 1, 0, None)
+    assert st == -6
+    st = _lib.gdn_step_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1, 64, 2, 64, 64, 0, 0, None)
+    assert st == -1
+    st = _lib.gdn_step_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, 2, 96, 64, 0, 0, None)
+    assert st == -5
