@@ -29,6 +29,7 @@ SIGNATURES = {
     "gdn_status_string": (ctypes.c_char_p, [_I]),
     "gdn_version": (ctypes.c_char_p, []),
     "gdn_launch_count": (ctypes.c_ulonglong, []),
+    "gdn_device_timeouts": (_I, [ctypes.POINTER(ctypes.c_uint)]),
     "gdn_set_kernel_timing": (None, [_I]),
     "gdn_read_kernel_timing": (_I, [ctypes.c_char_p, _I, ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(_I), _I]),
@@ -96,6 +97,15 @@ def gdn_status_string(status):
 
 def gdn_version():
     return load().gdn_version().decode()
+
+
+def gdn_device_timeouts():
+    """Bounded device-side waits that gave up on the current device (0 = none)."""
+    c = ctypes.c_uint(0)
+    st = load().gdn_device_timeouts(ctypes.byref(c))
+    if st != 0:
+        raise GDNError("gdn_device_timeouts", st)
+    return int(c.value)
 
 
 def gdn_launch_count():

@@ -1,15 +1,22 @@
 // gdn_api.cu -- the C-ABI entry points of libgdn.so: argument checks,
 // workspace planning and kernel dispatch.  See include/gdn.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/gdn.h"
 #include "common.cuh"
 #include "launch_stats.cuh"
 #include "simt_kernels.cuh"
+#include "tc_kernels.cuh"
+
+// Count of bounded device-side waits that gave up (see gdn_device_timeouts).
+static __device__ unsigned int g_wait_timeouts;
 
 namespace {
 
@@ -159,15 +166,118 @@ gdn_status dispatch_out(const Args &a, int bidir) {
                              : dispatch_dims<Tin, __nv_bfloat16>(a, bidir);
 }
 
-size_t plan_workspace(int B, int T, int H, int dk, int dv, int bidir) {
+// The tensor-core path takes bf16 inputs with d_k = 128; everything else runs
+// on the CUDA-core (fp32) path.
+bool use_tc(gdn_dtype dt, int dk, int dv) {
+    return dt == GDN_BF16 && dk == 128 && (dv == 128 || dv == 64);
+}
+
+size_t plan_workspace(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt, int bidir) {
     if (T == 0) return 0;
+    if (use_tc(dt, dk, dv))  // bidirectional with a bf16 output keeps an fp32 partial
+        return (bidir && o_dt == GDN_BF16) ? round_up((size_t)B * T * H * dv * sizeof(float), 256) : 0;
     return simt_workspace(B, T, H, dk, dv, bidir);
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core path
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tile map over a [B, T, H, d] bf16 tensor: boxes of (box_d columns, 1 head,
+// 64 tokens, 1 batch); tokens past T read as zero.
+bool encode_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, int box_d, bool swz128) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)box_d, 1, 64, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE,
+               swz128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+std::mutex g_err_mu;
+unsigned int *g_err_ptr[64] = {};
+
+unsigned int *timeout_counter() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> g(g_err_mu);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_wait_timeouts) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<unsigned int *>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+template <int DV, bool REV, typename Tout>
+gdn_status launch_tc(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq, const CUtensorMap &mv,
+                     const float *state_in, float *state_out, Tout *o, float *part, int out_mode,
+                     unsigned int *err) {
+    constexpr int NS = 32;
+    using SM = gdn::tc::Smem<NS>;
+    auto kern = gdn::tc::scan_kernel<DV, NS, REV, Tout>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const int nC = (a.T + kChunk - 1) / kChunk;
+    gdn::LaunchScope ls(REV ? "tc_scan_rev" : "tc_scan", a.stream);
+    kern<<<dim3(DV / NS, a.B * a.H), gdn::tc::kThreads, SM::kAlloc, a.stream>>>(
+        mk, mq, mv, a.alpha, a.beta, state_in, state_out, o, part, a.T, a.H, nC, out_mode, err);
+    return launch_status();
+}
+
+template <int DV, typename Tout>
+gdn_status run_tc(const Args &a, int bidir) {
+    using gdn::tc::kOutAddPartial;
+    using gdn::tc::kOutPartial;
+    using gdn::tc::kOutStore;
+    constexpr int NS = 32;
+    CUtensorMap mk, mq, mv;
+    if (!encode_map(&mk, a.k, a.B, a.T, a.H, 128, 64, true) ||
+        !encode_map(&mq, a.q, a.B, a.T, a.H, 128, 64, true) ||
+        !encode_map(&mv, a.v, a.B, a.T, a.H, DV, NS, false))
+        return GDN_ERR_CUDA;
+    unsigned int *err = timeout_counter();
+    if (!err) return GDN_ERR_CUDA;
+    Tout *o = static_cast<Tout *>(a.o);
+    if (!bidir)
+        return launch_tc<DV, false, Tout>(a, mk, mq, mv, a.state_in, a.state_out, o, nullptr, kOutStore, err);
+    // bidirectional: the causal pass writes (o, or an fp32 partial), the reverse pass adds
+    float *part = std::is_same<Tout, float>::value ? reinterpret_cast<float *>(a.o)
+                                                    : static_cast<float *>(a.ws);
+    const int first = std::is_same<Tout, float>::value ? kOutStore : kOutPartial;
+    gdn_status s = launch_tc<DV, false, Tout>(a, mk, mq, mv, nullptr, nullptr, o, part, first, err);
+    if (s != GDN_OK) return s;
+    return launch_tc<DV, true, Tout>(a, mk, mq, mv, nullptr, nullptr, o, part, kOutAddPartial, err);
+}
+
+gdn_status dispatch_tc(const Args &a, int bidir) {
+    if (a.dv == 128)
+        return a.o_dt == GDN_F32 ? run_tc<128, float>(a, bidir) : run_tc<128, __nv_bfloat16>(a, bidir);
+    return a.o_dt == GDN_F32 ? run_tc<64, float>(a, bidir) : run_tc<64, __nv_bfloat16>(a, bidir);
+}
+
 gdn_status run(const Args &a, int bidir) {
-    const gdn_status s = check_ws(a, plan_workspace(a.B, a.T, a.H, a.dk, a.dv, bidir));
+    const gdn_status s =
+        check_ws(a, plan_workspace(a.B, a.T, a.H, a.dk, a.dv, a.dt, a.o_dt, bidir));
     if (s != GDN_OK) return s;
     if (a.T == 0) return bidir ? GDN_OK : empty_scan(a);
+    if (use_tc(a.dt, a.dk, a.dv)) return dispatch_tc(a, bidir);
     return a.dt == GDN_F32 ? dispatch_out<float>(a, bidir) : dispatch_out<__nv_bfloat16>(a, bidir);
 }
 
@@ -248,7 +358,7 @@ gdn_status gdn_step_noalloc(const void *q, const void *k, const void *v, const f
            nullptr, 0, static_cast<cudaStream_t>(stream)};
     gdn_status s = check_common(a, T > 0);
     if (s != GDN_OK) return s;
-    const size_t need = plan_workspace(B, T, H, dk, dv, 0);
+    const size_t need = plan_workspace(B, T, H, dk, dv, dt, o_dt, 0);
     if (need > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
     if (need > 0) {
         s = noalloc_scratch(&a.ws);
@@ -263,7 +373,7 @@ size_t gdn_workspace_size(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn
     Args a{};
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.dt = dt; a.o_dt = o_dt;
     if (check_common(a, false) != GDN_OK) return 0;
-    return plan_workspace(B, T, H, dk, dv, bidir ? 1 : 0);
+    return plan_workspace(B, T, H, dk, dv, dt, o_dt, bidir ? 1 : 0);
 }
 
 const char *gdn_status_string(gdn_status s) {
@@ -281,6 +391,14 @@ const char *gdn_status_string(gdn_status s) {
 }
 
 const char *gdn_version(void) { return "gdn-b200 0.1 (sm_100a)"; }
+
+int gdn_device_timeouts(unsigned int *count) {
+    if (!count) return GDN_ERR_NULL;
+    unsigned int *p = timeout_counter();
+    if (!p) return GDN_ERR_CUDA;
+    return cudaMemcpy(count, p, sizeof(unsigned int), cudaMemcpyDeviceToHost) == cudaSuccess
+               ? GDN_OK : GDN_ERR_CUDA;
+}
 
 unsigned long long gdn_launch_count(void) {
     return gdn::LaunchStats::get().launches.load(std::memory_order_relaxed);

@@ -176,6 +176,11 @@ GDN_API const char *gdn_version(void);
  *   number of kernel names written, or a negative gdn_status.
  */
 GDN_API unsigned long long gdn_launch_count(void);
+/* gdn_device_timeouts -- number of bounded device-side waits (on TMA or
+ * tensor-core completion) that gave up on the current device since the
+ * library was loaded; non-zero means a kernel stopped early and its results
+ * are invalid.  Synchronous (reads a device word).  Returns a gdn_status. */
+GDN_API int gdn_device_timeouts(unsigned int *count);
 GDN_API void gdn_set_kernel_timing(int on);
 GDN_API int gdn_read_kernel_timing(char *names, int name_len, double *total_ms, int *launches,
                                    int max);

@@ -75,3 +75,9 @@ def test_rollout_168_steps():
     assert rel_err(o, o_one.float().cpu().numpy()) <= tol
     assert rel_err(state, s_one.cpu().numpy()) <= tol
     _check_heads(o.cpu(), inp, [5], s_gpu=state.cpu())
+
+
+def test_no_device_wait_gave_up():
+    """Every bounded device-side wait (TMA arrival, tensor-core completion) in
+    the kernels run so far completed in time."""
+    assert gdn.gdn_device_timeouts() == 0
