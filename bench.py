@@ -298,10 +298,16 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target length of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profiling aid: shorten T to this many tokens (not a benchmark result)")
     args = ap.parse_args()
 
+    import dataclasses
     from gated_delta_rule_72_b200 import inputs
     w = inputs.WORKLOADS[args.workload]
+    if args.tokens:
+        w = dataclasses.replace(w, T=min(w.T, args.tokens), name=w.name + "-T%d" % args.tokens)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -419,17 +425,9 @@ def main():
                  "frac": max(t_mem, t_flop) / (ms * 1e-3)}
 
     # ---- end to end through the public API, host buffers
-    pinned = {n: t.pin_memory() for n, t in step.host.items()}
-    dev_bufs = {n: torch.empty_like(t, device=device) for n, t in step.host.items()}
-    out_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
-    state_host = torch.empty(step.state.shape, dtype=torch.float32).pin_memory()
-    e2e_fn = lambda: step.run_e2e(pinned, dev_bufs, out_host, state_host)
-    for _ in range(2):
-        e2e_fn()
-    e2e_ms = timed(torch, e2e_fn, step.between, args.steps, dist)
-    e2e_ms = max_over_ranks(torch, dist, e2e_ms, device)
-    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = out_host.numel() * 4 + state_host.numel() * 4
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(torch, step, device, args, dist, units)
 
     # ---- oracle baseline on the host cores (rank 0, N = 1)
     cpu = None
@@ -445,16 +443,31 @@ def main():
                 "config": dict(config, l2=("inputs larger than L2, no flush" if step.flush is None
                                            else "L2 flushed between steps (256 MB write)")),
                 "roofline": roof, "step_roofline": step_roof,
-                "cpu_baseline": cpu,
-                "e2e": {"value": args.gpus * units / (e2e_ms * 1e-3) / 1e6, "unit": UNIT,
-                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                        "ms_per_step": e2e_ms},
-                "clocks": clocks, "gpu_launches": launches}
+                "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def run_e2e(torch, step, device, args, dist, units):
+    """Same metric end to end through the Python API: each step copies its
+    inputs from pinned host memory, runs the scan and reads back the output
+    and the final state, all inside the timed region."""
+    pinned = {n: t.pin_memory() for n, t in step.host.items()}
+    dev_bufs = {n: torch.empty_like(t, device=device) for n, t in step.host.items()}
+    out_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
+    state_host = torch.empty(step.state.shape, dtype=torch.float32).pin_memory()
+    e2e_fn = lambda: step.run_e2e(pinned, dev_bufs, out_host, state_host)
+    for _ in range(2):
+        e2e_fn()
+    e2e_ms = timed(torch, e2e_fn, step.between, args.steps, dist)
+    e2e_ms = max_over_ranks(torch, dist, e2e_ms, device)
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = out_host.numel() * 4 + state_host.numel() * 4
+    return {"value": args.gpus * units / (e2e_ms * 1e-3) / 1e6, "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
 
 if __name__ == "__main__":

@@ -13,7 +13,8 @@
 #include "common.cuh"
 #include "launch_stats.cuh"
 #include "simt_kernels.cuh"
-#include "tc_kernels.cuh"
+#include "tc_chain.cuh"
+#include "tc_prep.cuh"
 
 // Count of bounded device-side waits that gave up (see gdn_device_timeouts).
 static __device__ unsigned int g_wait_timeouts;
@@ -172,10 +173,20 @@ bool use_tc(gdn_dtype dt, int dk, int dv) {
     return dt == GDN_BF16 && dk == 128 && (dv == 128 || dv == 64);
 }
 
+size_t tc_record_bytes(int dv) {
+    return dv == 128 ? gdn::tc2::Rec<128>::kBytes : gdn::tc2::Rec<64>::kBytes;
+}
+
+// Tensor-core path workspace: one record per chunk, head and direction,
+// then (bidirectional with a bf16 output) an fp32 partial output.
 size_t plan_workspace(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt, int bidir) {
     if (T == 0) return 0;
-    if (use_tc(dt, dk, dv))  // bidirectional with a bf16 output keeps an fp32 partial
-        return (bidir && o_dt == GDN_BF16) ? round_up((size_t)B * T * H * dv * sizeof(float), 256) : 0;
+    if (use_tc(dt, dk, dv)) {
+        const size_t nC = (size_t)(T + kChunk - 1) / kChunk;
+        size_t bytes = round_up((bidir ? 2 : 1) * (size_t)B * H * nC * tc_record_bytes(dv), 256);
+        if (bidir && o_dt == GDN_BF16) bytes += round_up((size_t)B * T * H * dv * sizeof(float), 256);
+        return bytes;
+    }
     return simt_workspace(B, T, H, dk, dv, bidir);
 }
 
@@ -225,45 +236,73 @@ unsigned int *timeout_counter() {
     return g_err_ptr[dev];
 }
 
-template <int DV, bool REV, typename Tout>
-gdn_status launch_tc(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq, const CUtensorMap &mv,
-                     const float *state_in, float *state_out, Tout *o, float *part, int out_mode,
-                     unsigned int *err) {
-    constexpr int NS = 32;
-    using SM = gdn::tc::Smem<NS>;
-    auto kern = gdn::tc::scan_kernel<DV, NS, REV, Tout>;
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
+template <int DV>
+gdn_status launch_prep(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq, const CUtensorMap &mv,
+                       unsigned char *recs, int nC, int ndir, unsigned int *err) {
+    using SM = gdn::tc2::PrepSmem<DV>;
+    auto kern = gdn::tc2::prep_kernel<DV>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
         return GDN_ERR_CUDA;
-    const int nC = (a.T + kChunk - 1) / kChunk;
-    gdn::LaunchScope ls(REV ? "tc_scan_rev" : "tc_scan", a.stream);
-    kern<<<dim3(DV / NS, a.B * a.H), gdn::tc::kThreads, SM::kAlloc, a.stream>>>(
-        mk, mq, mv, a.alpha, a.beta, state_in, state_out, o, part, a.T, a.H, nC, out_mode, err);
+    const int nbh = a.B * a.H;
+    const long long ntasks = (long long)ndir * nC * nbh;
+    const int grid = (int)(ntasks < sm_count() ? ntasks : sm_count());
+    gdn::LaunchScope ls("tc_prep", a.stream);
+    kern<<<grid, gdn::tc2::kPrepThreads, SM::kAlloc, a.stream>>>(mk, mq, mv, a.alpha, a.beta, recs, a.T,
+                                                                 a.H, nC, nbh, 0, ndir, err);
+    return launch_status();
+}
+
+template <int DV, typename Tout>
+gdn_status launch_chain(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq,
+                        const unsigned char *recs, int nC, int dir, const float *state_in,
+                        float *state_out, Tout *o, float *part, int out_mode, unsigned int *err) {
+    constexpr int NS = 32;
+    using SM = gdn::tc2::ChainSmem<NS>;
+    auto kern = gdn::tc2::chain_kernel<DV, NS, Tout>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    gdn::LaunchScope ls(dir ? "tc_chain_rev" : "tc_chain", a.stream);
+    kern<<<dim3(DV / NS, a.B * a.H), gdn::tc2::kChainThreads, SM::kAlloc, a.stream>>>(
+        mk, mq, recs, state_in, state_out, o, part, a.T, a.H, nC, dir, out_mode, err);
     return launch_status();
 }
 
 template <int DV, typename Tout>
 gdn_status run_tc(const Args &a, int bidir) {
-    using gdn::tc::kOutAddPartial;
-    using gdn::tc::kOutPartial;
-    using gdn::tc::kOutStore;
-    constexpr int NS = 32;
+    using gdn::tc2::kOutAddPartial;
+    using gdn::tc2::kOutPartial;
+    using gdn::tc2::kOutStore;
     CUtensorMap mk, mq, mv;
     if (!encode_map(&mk, a.k, a.B, a.T, a.H, 128, 64, true) ||
         !encode_map(&mq, a.q, a.B, a.T, a.H, 128, 64, true) ||
-        !encode_map(&mv, a.v, a.B, a.T, a.H, DV, NS, false))
+        !encode_map(&mv, a.v, a.B, a.T, a.H, DV, 64, true))
         return GDN_ERR_CUDA;
     unsigned int *err = timeout_counter();
     if (!err) return GDN_ERR_CUDA;
+    const int nC = (a.T + kChunk - 1) / kChunk;
+    unsigned char *recs = static_cast<unsigned char *>(a.ws);
+    gdn_status s = launch_prep<DV>(a, mk, mq, mv, recs, nC, bidir ? 2 : 1, err);
+    if (s != GDN_OK) return s;
     Tout *o = static_cast<Tout *>(a.o);
     if (!bidir)
-        return launch_tc<DV, false, Tout>(a, mk, mq, mv, a.state_in, a.state_out, o, nullptr, kOutStore, err);
+        return launch_chain<DV, Tout>(a, mk, mq, recs, nC, 0, a.state_in, a.state_out, o, nullptr,
+                                      kOutStore, err);
     // bidirectional: the causal pass writes (o, or an fp32 partial), the reverse pass adds
+    const size_t rec_bytes = round_up(2 * (size_t)a.B * a.H * nC * tc_record_bytes(DV), 256);
     float *part = std::is_same<Tout, float>::value ? reinterpret_cast<float *>(a.o)
-                                                    : static_cast<float *>(a.ws);
+                                                    : reinterpret_cast<float *>(recs + rec_bytes);
     const int first = std::is_same<Tout, float>::value ? kOutStore : kOutPartial;
-    gdn_status s = launch_tc<DV, false, Tout>(a, mk, mq, mv, nullptr, nullptr, o, part, first, err);
+    s = launch_chain<DV, Tout>(a, mk, mq, recs, nC, 0, nullptr, nullptr, o, part, first, err);
     if (s != GDN_OK) return s;
-    return launch_tc<DV, true, Tout>(a, mk, mq, mv, nullptr, nullptr, o, part, kOutAddPartial, err);
+    return launch_chain<DV, Tout>(a, mk, mq, recs, nC, 1, nullptr, nullptr, o, part, kOutAddPartial, err);
 }
 
 gdn_status dispatch_tc(const Args &a, int bidir) {

@@ -1,0 +1,397 @@
+// tc_prep.cuh -- chunk preparation on the tensor cores (tcgen05 + TMA).
+//
+// For every chunk of 64 tokens of every (b, h) and direction (fully
+// parallel; a persistent grid walks the tasks and prefetches the next
+// task's tiles with TMA while it works on the current one) this kernel
+// computes, in the chunk's processing order r = 0..63 (the reverse direction
+// walks a chunk back to front):
+//   g_r = sum_{m<=r} log alpha_m                          (prefix sum, fp32)
+//   [K; Q] K^T                                            (kind::f16, M=128, exact)
+//   L_rs = beta_r e^{g_r-g_s} (KK^T)_rs, s < r             (fp32)
+//   P_rs = e^{g_r-g_s} (QK^T)_rs, s <= r   (forward)     | readout mask
+//        = e^{g_{r-1}-g_s} (QK^T)_rs, s < r (reverse)    |
+//   T = (I + L)^{-1}                                      (blocked 16x16, CUDA cores)
+//   W = T diag(beta e^g) K,  U = T diag(beta) V           (kind::f16, T as a hi/lo pair)
+//   dq_r = e^{g_r} (reverse: e^{g_{r-1}}),  dkk_r = e^{g_63 - g_r},  ds = e^{g_63}
+// and writes them as one record (tc_common.cuh) with rows in forward token
+// order: for the reverse direction every row and column index is mirrored
+// (r -> 63 - r), so that the chain kernel never needs to know the direction.
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace gdn {
+namespace tc2 {
+
+template <int DV>
+struct PrepSmem {
+    static constexpr int kKQ = 32768;                 // [K|Q] x 2 column blocks, 128B swizzle
+    static constexpr int kVb = 64 * DV * 2;           // V, 64-column blocks of 8 KB
+    static constexpr int kStage = kKQ + kVb;
+    static constexpr int kStage0 = 0;
+    static constexpr int kStage1 = kStage;            // both stages 1024-aligned
+    static constexpr int kL = 2 * kStage;             // [64][65] fp32
+    static constexpr int kT = kL + 64 * 65 * 4;       // [64][65] fp32
+    static constexpr int kX = kT + 64 * 65 * 4;       // 3 x [16][16] fp32
+    static constexpr int kT1h = (kX + 3 * 256 * 4 + 1023) / 1024 * 1024;
+    static constexpr int kT1l = kT1h + 8192;          // bf16 K-major 64 x 64
+    static constexpr int kT2h = kT1l + 8192;
+    static constexpr int kT2l = kT2h + 8192;
+    static constexpr int kGate = kT2l + 8192;         // g, beta, dq, dkk, beta e^g
+    static constexpr int kBar = kGate + 5 * 256;      // tma[2], mma
+    static constexpr int kCtl = kBar + 32;            // tmem base, abort, ds
+    static constexpr int kBytes = kCtl + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+    static_assert(kStage % 1024 == 0, "stages must stay 1024-aligned");
+    static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+constexpr int kPrepThreads = 256;
+constexpr uint32_t kPrepColG = 0;      // 128 lanes x 64
+constexpr uint32_t kPrepColW = 64;     // M=64 x 128
+constexpr uint32_t kPrepColU = 192;    // M=64 x DV
+constexpr uint32_t kPrepTmemCols = 512;
+
+// grid: persistent (<= tasks), block 256.  Tasks: dir-major, then chunk, then (b,h).
+template <int DV>
+__global__ void __launch_bounds__(kPrepThreads, 1)
+prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+            const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ alpha,
+            const float *__restrict__ beta, unsigned char *__restrict__ recs, int T, int H,
+            int nC, int nbh, int dir0, int ndir, unsigned int *__restrict__ err)
+{
+    using SM = PrepSmem<DV>;
+    using RC = Rec<DV>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    float *Lsm = reinterpret_cast<float *>(smem + SM::kL);
+    float *Tsm = reinterpret_cast<float *>(smem + SM::kT);
+    float *Xsm = reinterpret_cast<float *>(smem + SM::kX);
+    float *g_s = reinterpret_cast<float *>(smem + SM::kGate);
+    float *beta_s = g_s + 64;
+    float *dq_s = g_s + 128;
+    float *dkk_s = g_s + 192;
+    float *bg_s = g_s + 256;
+    uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + SM::kBar);   // [2]
+    uint64_t *mma_bar = tma_bar + 2;
+    uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + SM::kCtl);
+    volatile int *abort_s = reinterpret_cast<volatile int *>(smem + SM::kCtl + 4);
+    float *ds_s = reinterpret_cast<float *>(smem + SM::kCtl + 8);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3;                  // TMEM lane quarter of this warp
+    const int half = warp >> 2;                    // column half handled by this warp
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t sbase = smem_u32(smem);
+    const int ntasks = ndir * nC * nbh;
+
+    if (tid == 0) {
+        mbar_init(&tma_bar[0], 1);
+        mbar_init(&tma_bar[1], 1);
+        mbar_init(mma_bar, 1);
+        fence_mbar_init();
+        *abort_s = 0;
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_v);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_base_s, kPrepTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_s;
+
+    auto task_of = [&](int t, int &dir, int &c, int &bh) {
+        bh = t % nbh;
+        c = (t / nbh) % nC;
+        dir = dir0 + t / (nbh * nC);
+    };
+    auto issue_tma = [&](int t, int buf) {
+        int dir, c, bh;
+        task_of(t, dir, c, bh);
+        const int b = bh / H, h = bh % H, t0 = c * 64;
+        unsigned char *st = smem + (buf ? SM::kStage1 : SM::kStage0);
+        mbar_arrive_expect_tx(&tma_bar[buf], SM::kStage);
+        tma_load_4d(st, &tm_k, &tma_bar[buf], 0, h, t0, b);
+        tma_load_4d(st + 16384, &tm_k, &tma_bar[buf], 64, h, t0, b);
+        tma_load_4d(st + 8192, &tm_q, &tma_bar[buf], 0, h, t0, b);
+        tma_load_4d(st + 16384 + 8192, &tm_q, &tma_bar[buf], 64, h, t0, b);
+#pragma unroll
+        for (int vb = 0; vb < DV / 64; ++vb)
+            tma_load_4d(st + SM::kKQ + vb * 8192, &tm_v, &tma_bar[buf], vb * 64, h, t0, b);
+    };
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) {
+        if (!mbar_wait(bar, parity, kWaitTries)) {
+            *abort_s = 1;
+            if (err) atomicAdd(err, 1u);
+        }
+    };
+    // gates of a task, processing order: thread r < 64 loads row r
+    auto load_gates = [&](int t, float &la, float &bt) {
+        int dir, c, bh;
+        task_of(t, dir, c, bh);
+        const int b = bh / H, h = bh % H;
+        const int tok = token_of_row(c, tid, dir);
+        const size_t off = ((size_t)b * T + tok) * H + h;
+        la = tok < T ? __logf(alpha[off]) : 0.f;
+        bt = tok < T ? beta[off] : 0.f;
+    };
+
+    int t = blockIdx.x;
+    if (t < ntasks && tid == 0) issue_tma(t, 0);
+    float la_n = 0.f, bt_n = 0.f;
+    if (t < ntasks && tid < 64) load_gates(t, la_n, bt_n);
+    uint32_t tma_phases = 0, mma_phase = 0;   // bit b: parity of tma_bar[b]
+
+    for (int it = 0; t < ntasks; ++it, t += gridDim.x) {
+        const int buf = it & 1;
+        int dir, c, bh;
+        task_of(t, dir, c, bh);
+        const bool rev = dir != 0;
+        unsigned char *stage = smem + (buf ? SM::kStage1 : SM::kStage0);
+        const uint32_t st_addr = sbase + (buf ? SM::kStage1 : SM::kStage0);
+        unsigned char *rec = recs + ((size_t)(dir * nbh + bh) * nC + c) * RC::kBytes;
+
+        if (tid < 64) { g_s[tid] = la_n; beta_s[tid] = bt_n; }
+        wait_all(&tma_bar[buf], (tma_phases >> buf) & 1u);
+        tma_phases ^= 1u << buf;
+        __syncthreads();
+        if (*abort_s) break;
+        // prefetch the next task (its stage was released by the previous task's MMAs)
+        const int tn = t + gridDim.x;
+        if (tn < ntasks) {
+            if (tid == 0) issue_tma(tn, buf ^ 1);
+            if (tid < 64) load_gates(tn, la_n, bt_n);
+        }
+        if (warp == 0) {  // inclusive prefix sum of log alpha, 2 rows per lane
+            const float a0 = g_s[2 * lane], a1 = g_s[2 * lane + 1];
+            float s = a0 + a1;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, s, d);
+                if (lane >= d) s += y;
+            }
+            const float ex = s - (a0 + a1);
+            g_s[2 * lane] = ex + a0;
+            g_s[2 * lane + 1] = ex + a0 + a1;
+        }
+        __syncthreads();
+        if (tid < 64) {
+            const float gr = g_s[tid], gl = g_s[63];
+            dq_s[tid] = rev ? (tid > 0 ? __expf(g_s[tid - 1]) : 1.f) : __expf(gr);
+            dkk_s[tid] = __expf(gl - gr);
+            bg_s[tid] = beta_s[tid] * __expf(gr);
+            if (tid == 0) *ds_s = __expf(gl);
+        }
+        // ---- [K; Q] K^T -------------------------------------------------------
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t id = idesc(128, 64, 1, 0, 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t a = st_addr + (s >> 2) * 16384 + (s & 3) * 32;
+                mma_bf16(tmem + kPrepColG, sdesc_sw128(a), sdesc_sw128(a), id, s > 0);
+            }
+            mma_commit(mma_bar);
+        }
+        wait_all(mma_bar, mma_phase);
+        mma_phase ^= 1;
+        tc_fence_after();
+        __syncthreads();  // gate vectors ready
+        // ---- L (fp32, to shared) and P (hi/lo, to the record) ------------------------
+        {
+            float G[32];
+            tmem_ld16(tmem + lane_base + kPrepColG + half * 32, G);
+            tmem_ld16(tmem + lane_base + kPrepColG + half * 32 + 16, G + 16);
+            tmem_wait_ld();
+            const int ln = quarter * 32 + lane;          // TMEM lane = Gram row
+            const int fl = ln & 63;                      // forward row within the chunk
+            const int r = rev ? 63 - fl : fl;            // processing row
+            const int f0 = half * 32;                    // forward columns f0 .. f0+31
+            if (ln < 64) {
+                const float br = beta_s[r], gr = g_s[r];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int s = rev ? 63 - (f0 + e) : f0 + e;
+                    Lsm[r * 65 + s] = s < r ? br * __expf(gr - g_s[s]) * G[e] : 0.f;
+                }
+            } else {
+                const float gq = rev ? (r > 0 ? g_s[r - 1] : 0.f) : g_s[r];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int f = f0 + cc * 8 + e;
+                        const int s = rev ? 63 - f : f;
+                        const bool keep = rev ? (s < r) : (s <= r);
+                        v[e] = keep ? __expf(gq - g_s[s]) * G[cc * 8 + e] : 0.f;
+                    }
+                    uint4 hi, lo;
+                    split2(v[0], v[1], hi.x, lo.x);
+                    split2(v[2], v[3], hi.y, lo.y);
+                    split2(v[4], v[5], hi.z, lo.z);
+                    split2(v[6], v[7], hi.w, lo.w);
+                    const int off = kmaj64(fl, f0 + cc * 8);
+                    *reinterpret_cast<uint4 *>(rec + RC::kPh + off) = hi;
+                    *reinterpret_cast<uint4 *>(rec + RC::kPl + off) = lo;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        // ---- T = (I + L)^{-1}, blocked 16 x 16 (processing order) ------------------
+        if (tid < 64) {
+            const int blk = tid >> 4, j = tid & 15, o0 = blk * 16;
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float acc = (i == j) ? 1.f : 0.f;
+#pragma unroll
+                for (int m = 0; m < i; ++m) acc = fmaf(-Lsm[(o0 + i) * 65 + o0 + m], x[m], acc);
+                x[i] = acc;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) Tsm[(o0 + i) * 65 + o0 + j] = x[i];
+        } else {
+            for (int e = tid - 64; e < 64 * 64; e += kPrepThreads - 64) {
+                const int i = e >> 6, jj = e & 63;
+                if ((jj >> 4) > (i >> 4)) Tsm[i * 65 + jj] = 0.f;
+            }
+        }
+        __syncthreads();
+        for (int band = 1; band < 4; ++band) {
+            const int nblk = 4 - band;
+            for (int e = tid; e < nblk * 256; e += kPrepThreads) {
+                const int j = e >> 8, ii = (e >> 4) & 15, jj = e & 15;
+                const int i = j + band;
+                float acc = 0.f;
+                for (int k = j; k < i; ++k) {
+#pragma unroll
+                    for (int m = 0; m < 16; ++m)
+                        acc = fmaf(Lsm[(i * 16 + ii) * 65 + k * 16 + m], Tsm[(k * 16 + m) * 65 + j * 16 + jj], acc);
+                }
+                Xsm[j * 256 + ii * 16 + jj] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < nblk * 256; e += kPrepThreads) {
+                const int j = e >> 8, ii = (e >> 4) & 15, jj = e & 15;
+                const int i = j + band;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    acc = fmaf(Tsm[(i * 16 + ii) * 65 + i * 16 + m], Xsm[j * 256 + m * 16 + jj], acc);
+                Tsm[(i * 16 + ii) * 65 + j * 16 + jj] = -acc;
+            }
+            __syncthreads();
+        }
+        // ---- A operands T diag(beta e^g) and T diag(beta) as hi/lo pairs, in forward
+        //      row/column order (mirrored for the reverse direction) -----------------
+        for (int cell = tid; cell < 64 * 8; cell += kPrepThreads) {
+            const int fr = cell & 63, fc0 = (cell >> 6) * 8;
+            const int r = rev ? 63 - fr : fr;
+            float a[8], bvals[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int s = rev ? 63 - (fc0 + e) : fc0 + e;
+                const float tv = Tsm[r * 65 + s];
+                a[e] = tv * bg_s[s];
+                bvals[e] = tv * beta_s[s];
+            }
+            uint4 h1, l1, h2, l2;
+            split2(a[0], a[1], h1.x, l1.x); split2(a[2], a[3], h1.y, l1.y);
+            split2(a[4], a[5], h1.z, l1.z); split2(a[6], a[7], h1.w, l1.w);
+            split2(bvals[0], bvals[1], h2.x, l2.x); split2(bvals[2], bvals[3], h2.y, l2.y);
+            split2(bvals[4], bvals[5], h2.z, l2.z); split2(bvals[6], bvals[7], h2.w, l2.w);
+            const int off = kmaj64(fr, fc0);
+            *reinterpret_cast<uint4 *>(smem + SM::kT1h + off) = h1;
+            *reinterpret_cast<uint4 *>(smem + SM::kT1l + off) = l1;
+            *reinterpret_cast<uint4 *>(smem + SM::kT2h + off) = h2;
+            *reinterpret_cast<uint4 *>(smem + SM::kT2l + off) = l2;
+        }
+        fence_async_shared();
+        __syncthreads();
+        // ---- W = T1 K and U = T2 V on the tensor cores (K and V straight from the tiles)
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idw = idesc(64, 128, 1, 0, 1);
+            constexpr uint32_t idu = idesc(64, DV, 1, 0, 1);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t t1 = sbase + (part ? SM::kT1l : SM::kT1h);
+                const uint32_t t2 = sbase + (part ? SM::kT2l : SM::kT2h);
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const uint32_t acc = (part | s) != 0;
+                    mma_bf16(tmem + kPrepColW, sdesc_noswz(t1 + 2 * s * 1024, 1024, 128),
+                             sdesc_sw128_mn(st_addr + s * 2048, 16384), idw, acc);
+                    mma_bf16(tmem + kPrepColU, sdesc_noswz(t2 + 2 * s * 1024, 1024, 128),
+                             sdesc_sw128_mn(st_addr + SM::kKQ + s * 2048, 8192), idu, acc);
+                }
+            }
+            mma_commit(mma_bar);
+        }
+        wait_all(mma_bar, mma_phase);
+        mma_phase ^= 1;
+        tc_fence_after();
+        // ---- record: W (bf16 image), U (fp32 rows), gate vectors ------------------
+        {
+            const bool row_lane = lane < 16;
+            const int f = quarter * 16 + lane;       // forward row (M=64 accumulator layout)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {            // W columns half*64 .. +63
+                float w[16];
+                tmem_ld16(tmem + lane_base + kPrepColW + half * 64 + q * 16, w);
+                tmem_wait_ld();
+                if (row_lane) {
+                    uint4 p0, p1;
+                    p0.x = pack_bf16(w[0], w[1]); p0.y = pack_bf16(w[2], w[3]);
+                    p0.z = pack_bf16(w[4], w[5]); p0.w = pack_bf16(w[6], w[7]);
+                    p1.x = pack_bf16(w[8], w[9]); p1.y = pack_bf16(w[10], w[11]);
+                    p1.z = pack_bf16(w[12], w[13]); p1.w = pack_bf16(w[14], w[15]);
+                    const int d0 = half * 64 + q * 16;
+                    *reinterpret_cast<uint4 *>(rec + RC::kW + (d0 >> 3) * 1024 + f * 16) = p0;
+                    *reinterpret_cast<uint4 *>(rec + RC::kW + ((d0 + 8) >> 3) * 1024 + f * 16) = p1;
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < DV / 32; ++q) {      // U columns half*DV/2 .. +DV/2-1
+                float u[16];
+                const int col = half * (DV / 2) + q * 16;
+                tmem_ld16(tmem + lane_base + kPrepColU + col, u);
+                tmem_wait_ld();
+                if (row_lane) {
+                    float4 *dst = reinterpret_cast<float4 *>(rec + RC::kU + (f * DV + col) * 4);
+                    dst[0] = make_float4(u[0], u[1], u[2], u[3]);
+                    dst[1] = make_float4(u[4], u[5], u[6], u[7]);
+                    dst[2] = make_float4(u[8], u[9], u[10], u[11]);
+                    dst[3] = make_float4(u[12], u[13], u[14], u[15]);
+                }
+            }
+            if (tid < 64) {
+                const int r = rev ? 63 - tid : tid;   // record row tid <- processing row r
+                float *gate = reinterpret_cast<float *>(rec + RC::kGate);
+                gate[tid] = dq_s[r];
+                gate[64 + tid] = dkk_s[r];
+                if (tid == 0) gate[128] = *ds_s;
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    if (*abort_s) {
+        mbar_wait(&tma_bar[0], tma_phases & 1u, 1u << 16);
+        mbar_wait(&tma_bar[1], (tma_phases >> 1) & 1u, 1u << 16);
+        mbar_wait(mma_bar, mma_phase, 1u << 16);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kPrepTmemCols);
+}
+
+}  // namespace tc2
+}  // namespace gdn
