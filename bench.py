@@ -124,7 +124,7 @@ class ClockSampler:
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + SMI_FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -371,10 +371,14 @@ def main():
     # ---- the timed region: K steps, per-kernel events on, clocks sampled
     sampler = ClockSampler(range(args.gpus)) if rank == 0 else None
     if sampler:
+        # nvidia-smi takes a moment to start sampling: keep the GPU busy with
+        # extra untimed steps for ~1 s so samples cover the load up to the
+        # timed region, which follows immediately
         sampler.start()
-        time.sleep(0.3)
-        for _ in range(2):       # keep the GPU busy while nvidia-smi starts
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
             step.run()
+            torch.cuda.synchronize()
     gdn.gdn_read_kernel_timing()                  # drop anything recorded so far
     n0 = gdn.gdn_launch_count()
     gdn.gdn_set_kernel_timing(1)

@@ -253,7 +253,8 @@ gdn_status launch_prep(const Args &a, const CUtensorMap &mk, const CUtensorMap &
         return GDN_ERR_CUDA;
     const int nbh = a.B * a.H;
     const long long ntasks = (long long)ndir * nC * nbh;
-    const int grid = (int)(ntasks < sm_count() ? ntasks : sm_count());
+    const long long slots = (long long)sm_count() * gdn::tc2::kPrepCtasPerSm;
+    const int grid = (int)(ntasks < slots ? ntasks : slots);
     gdn::LaunchScope ls("tc_prep", a.stream);
     kern<<<grid, gdn::tc2::kPrepThreads, SM::kAlloc, a.stream>>>(mk, mq, mv, a.alpha, a.beta, recs, a.T,
                                                                  a.H, nC, nbh, 0, ndir, err);

@@ -21,7 +21,10 @@ namespace tc2 {
 using namespace gdn::sm100;
 
 constexpr int kDK = 128;                     // key dimension of the tensor-core path
-constexpr uint32_t kWaitTries = 1u << 22;    // bounded mbarrier polls
+constexpr uint32_t kWaitTries = 1u << 24;    // bounded mbarrier polls
+
+// Width of the state slice one chain CTA owns (columns of d_v).
+constexpr int kSliceCols = 32;
 
 // Per-chunk record written by the prep kernel and read by the chain kernel,
 // rows in FORWARD token order for either direction (the reverse direction's
@@ -29,15 +32,18 @@ constexpr uint32_t kWaitTries = 1u << 22;    // bounded mbarrier polls
 //   W   bf16, K-major no-swizzle A operand, 64 rows x 128 (d_k)   16384 B
 //   Ph  bf16, K-major no-swizzle A operand, 64 x 64                8192 B
 //   Pl  bf16, same layout (P - Ph)                                 8192 B
-//   U   fp32 row-major [64][DV]                                    256*DV B
+//   U   fp32, slice-major [DV/32][64][32] (one slice contiguous)   256*DV B
 //   dq[64], dkk[64], ds, padding                                   1024 B
+// so that a chain CTA fetches its operands with a handful of bulk copies.
 template <int DV>
 struct Rec {
     static constexpr int kW = 0;
     static constexpr int kPh = 16384;
     static constexpr int kPl = 24576;
     static constexpr int kU = 32768;
+    static constexpr int kUSlice = 64 * kSliceCols * 4;     // bytes of one slice of U
     static constexpr int kGate = kU + 64 * DV * 4;
+    static constexpr int kGateCopy = 528;                   // dq, dkk, ds rounded to 16 bytes
     static constexpr int kBytes = kGate + 1024;
 };
 

@@ -1,8 +1,8 @@
 // tc_prep.cuh -- chunk preparation on the tensor cores (tcgen05 + TMA).
 //
 // For every chunk of 64 tokens of every (b, h) and direction (fully
-// parallel; a persistent grid walks the tasks and prefetches the next
-// task's tiles with TMA while it works on the current one) this kernel
+// parallel; a persistent grid of two CTAs per SM walks the tasks and fetches
+// the next task's tiles with TMA while it finishes the current one) this kernel
 // computes, in the chunk's processing order r = 0..63 (the reverse direction
 // walks a chunk back to front):
 //   g_r = sum_{m<=r} log alpha_m                          (prefix sum, fp32)
@@ -11,7 +11,8 @@
 //   P_rs = e^{g_r-g_s} (QK^T)_rs, s <= r   (forward)     | readout mask
 //        = e^{g_{r-1}-g_s} (QK^T)_rs, s < r (reverse)    |
 //   T = (I + L)^{-1}                                      (blocked 16x16, CUDA cores)
-//   W = T diag(beta e^g) K,  U = T diag(beta) V           (kind::f16, T as a hi/lo pair)
+//   W = T diag(beta e^g) K,  U = T diag(beta) V           (kind::f16; the T of U as a
+//                                                          hi/lo pair, W rounds to bf16 anyway)
 //   dq_r = e^{g_r} (reverse: e^{g_{r-1}}),  dkk_r = e^{g_63 - g_r},  ds = e^{g_63}
 // and writes them as one record (tc_common.cuh) with rows in forward token
 // order: for the reverse direction every row and column index is mirrored
@@ -27,34 +28,32 @@ template <int DV>
 struct PrepSmem {
     static constexpr int kKQ = 32768;                 // [K|Q] x 2 column blocks, 128B swizzle
     static constexpr int kVb = 64 * DV * 2;           // V, 64-column blocks of 8 KB
-    static constexpr int kStage = kKQ + kVb;
-    static constexpr int kStage0 = 0;
-    static constexpr int kStage1 = kStage;            // both stages 1024-aligned
-    static constexpr int kL = 2 * kStage;             // [64][65] fp32
+    static constexpr int kStage = kKQ + kVb;          // one stage, 1024-aligned
+    static constexpr int kL = kStage;                 // [64][65] fp32
     static constexpr int kT = kL + 64 * 65 * 4;       // [64][65] fp32
     static constexpr int kX = kT + 64 * 65 * 4;       // 3 x [16][16] fp32
-    static constexpr int kT1h = (kX + 3 * 256 * 4 + 1023) / 1024 * 1024;
-    static constexpr int kT1l = kT1h + 8192;          // bf16 K-major 64 x 64
-    static constexpr int kT2h = kT1l + 8192;
+    static constexpr int kT1 = (kX + 3 * 256 * 4 + 1023) / 1024 * 1024;   // bf16 K-major 64 x 64
+    static constexpr int kT2h = kT1 + 8192;
     static constexpr int kT2l = kT2h + 8192;
     static constexpr int kGate = kT2l + 8192;         // g, beta, dq, dkk, beta e^g
-    static constexpr int kBar = kGate + 5 * 256;      // tma[2], mma
-    static constexpr int kCtl = kBar + 32;            // tmem base, abort, ds
+    static constexpr int kBar = kGate + 5 * 256;      // tma, mma
+    static constexpr int kCtl = kBar + 16;            // tmem base, abort, ds
     static constexpr int kBytes = kCtl + 16;
     static constexpr int kAlloc = kBytes + 1024;
-    static_assert(kStage % 1024 == 0, "stages must stay 1024-aligned");
-    static_assert(kAlloc <= 232448, "shared memory budget");
+    static_assert(kStage % 1024 == 0, "the stage must stay 1024-aligned");
+    static_assert(kAlloc <= 232448 / 2 - 1024, "two CTAs per SM");
 };
 
 constexpr int kPrepThreads = 256;
-constexpr uint32_t kPrepColG = 0;      // 128 lanes x 64
-constexpr uint32_t kPrepColW = 64;     // M=64 x 128
-constexpr uint32_t kPrepColU = 192;    // M=64 x DV
-constexpr uint32_t kPrepTmemCols = 512;
+constexpr int kPrepCtasPerSm = 2;
+constexpr uint32_t kPrepColG = 0;      // 128 lanes x 64 (dead before W is written)
+constexpr uint32_t kPrepColW = 0;      // M=64 x 128
+constexpr uint32_t kPrepColU = 128;    // M=64 x DV
+constexpr uint32_t kPrepTmemCols = 256;
 
 // grid: persistent (<= tasks), block 256.  Tasks: dir-major, then chunk, then (b,h).
 template <int DV>
-__global__ void __launch_bounds__(kPrepThreads, 1)
+__global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
 prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
             const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ alpha,
             const float *__restrict__ beta, unsigned char *__restrict__ recs, int T, int H,
@@ -72,8 +71,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     float *dq_s = g_s + 128;
     float *dkk_s = g_s + 192;
     float *bg_s = g_s + 256;
-    uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + SM::kBar);   // [2]
-    uint64_t *mma_bar = tma_bar + 2;
+    uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + SM::kBar);
+    uint64_t *mma_bar = tma_bar + 1;
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + SM::kCtl);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + SM::kCtl + 4);
     float *ds_s = reinterpret_cast<float *>(smem + SM::kCtl + 8);
@@ -86,8 +85,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     const int ntasks = ndir * nC * nbh;
 
     if (tid == 0) {
-        mbar_init(&tma_bar[0], 1);
-        mbar_init(&tma_bar[1], 1);
+        mbar_init(tma_bar, 1);
         mbar_init(mma_bar, 1);
         fence_mbar_init();
         *abort_s = 0;
@@ -109,19 +107,19 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         c = (t / nbh) % nC;
         dir = dir0 + t / (nbh * nC);
     };
-    auto issue_tma = [&](int t, int buf) {
+    auto issue_tma = [&](int t) {
         int dir, c, bh;
         task_of(t, dir, c, bh);
         const int b = bh / H, h = bh % H, t0 = c * 64;
-        unsigned char *st = smem + (buf ? SM::kStage1 : SM::kStage0);
-        mbar_arrive_expect_tx(&tma_bar[buf], SM::kStage);
-        tma_load_4d(st, &tm_k, &tma_bar[buf], 0, h, t0, b);
-        tma_load_4d(st + 16384, &tm_k, &tma_bar[buf], 64, h, t0, b);
-        tma_load_4d(st + 8192, &tm_q, &tma_bar[buf], 0, h, t0, b);
-        tma_load_4d(st + 16384 + 8192, &tm_q, &tma_bar[buf], 64, h, t0, b);
+        unsigned char *st = smem;
+        mbar_arrive_expect_tx(tma_bar, SM::kStage);
+        tma_load_4d(st, &tm_k, tma_bar, 0, h, t0, b);
+        tma_load_4d(st + 16384, &tm_k, tma_bar, 64, h, t0, b);
+        tma_load_4d(st + 8192, &tm_q, tma_bar, 0, h, t0, b);
+        tma_load_4d(st + 16384 + 8192, &tm_q, tma_bar, 64, h, t0, b);
 #pragma unroll
         for (int vb = 0; vb < DV / 64; ++vb)
-            tma_load_4d(st + SM::kKQ + vb * 8192, &tm_v, &tma_bar[buf], vb * 64, h, t0, b);
+            tma_load_4d(st + SM::kKQ + vb * 8192, &tm_v, tma_bar, vb * 64, h, t0, b);
     };
     auto wait_all = [&](uint64_t *bar, uint32_t parity) {
         if (!mbar_wait(bar, parity, kWaitTries)) {
@@ -141,31 +139,25 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     };
 
     int t = blockIdx.x;
-    if (t < ntasks && tid == 0) issue_tma(t, 0);
+    if (t < ntasks && tid == 0) issue_tma(t);
     float la_n = 0.f, bt_n = 0.f;
     if (t < ntasks && tid < 64) load_gates(t, la_n, bt_n);
-    uint32_t tma_phases = 0, mma_phase = 0;   // bit b: parity of tma_bar[b]
+    uint32_t tma_phase = 0, mma_phase = 0;
+    const uint32_t st_addr = sbase;
 
-    for (int it = 0; t < ntasks; ++it, t += gridDim.x) {
-        const int buf = it & 1;
+    for (; t < ntasks; t += gridDim.x) {
         int dir, c, bh;
         task_of(t, dir, c, bh);
         const bool rev = dir != 0;
-        unsigned char *stage = smem + (buf ? SM::kStage1 : SM::kStage0);
-        const uint32_t st_addr = sbase + (buf ? SM::kStage1 : SM::kStage0);
         unsigned char *rec = recs + ((size_t)(dir * nbh + bh) * nC + c) * RC::kBytes;
+        const int tn = t + gridDim.x;
 
         if (tid < 64) { g_s[tid] = la_n; beta_s[tid] = bt_n; }
-        wait_all(&tma_bar[buf], (tma_phases >> buf) & 1u);
-        tma_phases ^= 1u << buf;
+        wait_all(tma_bar, tma_phase);
+        tma_phase ^= 1;
         __syncthreads();
         if (*abort_s) break;
-        // prefetch the next task (its stage was released by the previous task's MMAs)
-        const int tn = t + gridDim.x;
-        if (tn < ntasks) {
-            if (tid == 0) issue_tma(tn, buf ^ 1);
-            if (tid < 64) load_gates(tn, la_n, bt_n);
-        }
+        if (tn < ntasks && tid < 64) load_gates(tn, la_n, bt_n);   // next task's gates travel meanwhile
         if (warp == 0) {  // inclusive prefix sum of log alpha, 2 rows per lane
             const float a0 = g_s[2 * lane], a1 = g_s[2 * lane + 1];
             float s = a0 + a1;
@@ -288,8 +280,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             }
             __syncthreads();
         }
-        // ---- A operands T diag(beta e^g) and T diag(beta) as hi/lo pairs, in forward
-        //      row/column order (mirrored for the reverse direction) -----------------
+        // ---- A operands T diag(beta e^g) (bf16) and T diag(beta) (hi/lo pair), in
+        //      forward row/column order (mirrored for the reverse direction) --------
         for (int cell = tid; cell < 64 * 8; cell += kPrepThreads) {
             const int fr = cell & 63, fc0 = (cell >> 6) * 8;
             const int r = rev ? 63 - fr : fr;
@@ -301,14 +293,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 a[e] = tv * bg_s[s];
                 bvals[e] = tv * beta_s[s];
             }
-            uint4 h1, l1, h2, l2;
-            split2(a[0], a[1], h1.x, l1.x); split2(a[2], a[3], h1.y, l1.y);
-            split2(a[4], a[5], h1.z, l1.z); split2(a[6], a[7], h1.w, l1.w);
+            uint4 h1, h2, l2;
+            h1.x = pack_bf16(a[0], a[1]); h1.y = pack_bf16(a[2], a[3]);
+            h1.z = pack_bf16(a[4], a[5]); h1.w = pack_bf16(a[6], a[7]);
             split2(bvals[0], bvals[1], h2.x, l2.x); split2(bvals[2], bvals[3], h2.y, l2.y);
             split2(bvals[4], bvals[5], h2.z, l2.z); split2(bvals[6], bvals[7], h2.w, l2.w);
             const int off = kmaj64(fr, fc0);
-            *reinterpret_cast<uint4 *>(smem + SM::kT1h + off) = h1;
-            *reinterpret_cast<uint4 *>(smem + SM::kT1l + off) = l1;
+            *reinterpret_cast<uint4 *>(smem + SM::kT1 + off) = h1;
             *reinterpret_cast<uint4 *>(smem + SM::kT2h + off) = h2;
             *reinterpret_cast<uint4 *>(smem + SM::kT2l + off) = l2;
         }
@@ -320,23 +311,22 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             constexpr uint32_t idw = idesc(64, 128, 1, 0, 1);
             constexpr uint32_t idu = idesc(64, DV, 1, 0, 1);
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t t1 = sbase + (part ? SM::kT1l : SM::kT1h);
-                const uint32_t t2 = sbase + (part ? SM::kT2l : SM::kT2h);
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const uint32_t acc = (part | s) != 0;
-                    mma_bf16(tmem + kPrepColW, sdesc_noswz(t1 + 2 * s * 1024, 1024, 128),
-                             sdesc_sw128_mn(st_addr + s * 2048, 16384), idw, acc);
-                    mma_bf16(tmem + kPrepColU, sdesc_noswz(t2 + 2 * s * 1024, 1024, 128),
-                             sdesc_sw128_mn(st_addr + SM::kKQ + s * 2048, 8192), idu, acc);
-                }
+            for (int s = 0; s < 4; ++s) {
+                mma_bf16(tmem + kPrepColW, sdesc_noswz(sbase + SM::kT1 + 2 * s * 1024, 1024, 128),
+                         sdesc_sw128_mn(st_addr + s * 2048, 16384), idw, s > 0);
+                const uint64_t bv = sdesc_sw128_mn(st_addr + SM::kKQ + s * 2048, 8192);
+                mma_bf16(tmem + kPrepColU, sdesc_noswz(sbase + SM::kT2h + 2 * s * 1024, 1024, 128),
+                         bv, idu, s > 0);
+                mma_bf16(tmem + kPrepColU, sdesc_noswz(sbase + SM::kT2l + 2 * s * 1024, 1024, 128),
+                         bv, idu, 1);
             }
             mma_commit(mma_bar);
         }
         wait_all(mma_bar, mma_phase);
         mma_phase ^= 1;
         tc_fence_after();
+        // the tiles are consumed: fetch the next task's while this one is written out
+        if (tn < ntasks && tid == 0) issue_tma(tn);
         // ---- record: W (bf16 image), U (fp32 rows), gate vectors ------------------
         {
             const bool row_lane = lane < 16;
@@ -363,8 +353,9 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 const int col = half * (DV / 2) + q * 16;
                 tmem_ld16(tmem + lane_base + kPrepColU + col, u);
                 tmem_wait_ld();
-                if (row_lane) {
-                    float4 *dst = reinterpret_cast<float4 *>(rec + RC::kU + (f * DV + col) * 4);
+                if (row_lane) {   // slice-major: slice col/32, row f, columns col%32 ..
+                    float4 *dst = reinterpret_cast<float4 *>(
+                        rec + RC::kU + (col / kSliceCols) * RC::kUSlice + (f * kSliceCols + col % kSliceCols) * 4);
                     dst[0] = make_float4(u[0], u[1], u[2], u[3]);
                     dst[1] = make_float4(u[4], u[5], u[6], u[7]);
                     dst[2] = make_float4(u[8], u[9], u[10], u[11]);
@@ -384,9 +375,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     }
 
     if (*abort_s) {
-        mbar_wait(&tma_bar[0], tma_phases & 1u, 1u << 16);
-        mbar_wait(&tma_bar[1], (tma_phases >> 1) & 1u, 1u << 16);
-        mbar_wait(mma_bar, mma_phase, 1u << 16);
+        mbar_wait(tma_bar, tma_phase, 64);
+        mbar_wait(mma_bar, mma_phase, 64);
     }
     tc_fence_before();
     __syncthreads();
