@@ -177,14 +177,24 @@ size_t tc_record_bytes(int dv) {
     return dv == 128 ? gdn::tc2::Rec<128>::kBytes : gdn::tc2::Rec<64>::kBytes;
 }
 
-// Tensor-core path workspace: one record per chunk, head and direction,
-// then (bidirectional with a bf16 output) an fp32 partial output.
+// Tensor-core path workspace: one record per chunk, head and direction; then,
+// bidirectional only, the fp32 output piece buffers of the two directions
+// (the causal one is o itself when o is fp32) and one counter per piece.
+size_t tc_pair_counters(int B, int T, int H, int dv) {
+    const size_t nC = (size_t)(T + kChunk - 1) / kChunk;
+    return (size_t)B * H * nC * (dv / gdn::tc2::kChainNS) * 8;
+}
+
 size_t plan_workspace(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt, int bidir) {
     if (T == 0) return 0;
     if (use_tc(dt, dk, dv)) {
         const size_t nC = (size_t)(T + kChunk - 1) / kChunk;
         size_t bytes = round_up((bidir ? 2 : 1) * (size_t)B * H * nC * tc_record_bytes(dv), 256);
-        if (bidir && o_dt == GDN_BF16) bytes += round_up((size_t)B * T * H * dv * sizeof(float), 256);
+        if (bidir) {
+            const size_t part = round_up((size_t)B * T * H * dv * sizeof(float), 256);
+            bytes += (o_dt == GDN_BF16 ? 2 : 1) * part;
+            bytes += round_up(tc_pair_counters(B, T, H, dv) * sizeof(unsigned int), 256);
+        }
         return bytes;
     }
     return simt_workspace(B, T, H, dk, dv, bidir);
@@ -206,17 +216,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// Tile map over a [B, T, H, d] bf16 tensor: boxes of (box_d columns, 1 head,
-// 64 tokens, 1 batch); tokens past T read as zero.
-bool encode_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, int box_d, bool swz128) {
+// Tile map over a [B, T, H, d] tensor of bf16 (esize 2) or fp32 (esize 4):
+// boxes of (box_d columns, 1 head, 64 tokens, 1 batch); loads past T read as
+// zero and stores past T are dropped.
+bool encode_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, int box_d, bool swz128,
+                int esize = 2) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) return false;
+    const cuuint64_t es = (cuuint64_t)esize;
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)H * d * es, (cuuint64_t)T * H * d * es};
     const cuuint32_t box[4] = {(cuuint32_t)box_d, 1, 64, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE,
+    return enc(m, esize == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                swz128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -263,24 +276,20 @@ gdn_status launch_prep(const Args &a, const CUtensorMap &mk, const CUtensorMap &
 
 template <int DV, typename Tout>
 gdn_status launch_chain(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq,
-                        const unsigned char *recs, int nC, int dir, const float *state_in,
-                        float *state_out, Tout *o, float *part, int out_mode, unsigned int *err) {
-    constexpr int NS = 32;
-    using SM = gdn::tc2::ChainSmem<NS>;
-    auto kern = gdn::tc2::chain_kernel<DV, NS, Tout>;
+                        const CUtensorMap &mo, const unsigned char *recs, int nC, int ndir, const float *state_in,
+                        float *state_out, const gdn::tc2::ChainOut<Tout> &out, unsigned int *err) {
+    using SM = gdn::tc2::ChainSmem;
+    auto kern = gdn::tc2::chain_kernel<DV, Tout>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
         return GDN_ERR_CUDA;
-    gdn::LaunchScope ls(dir ? "tc_chain_rev" : "tc_chain", a.stream);
-    kern<<<dim3(DV / NS, a.B * a.H), gdn::tc2::kChainThreads, SM::kAlloc, a.stream>>>(
-        mk, mq, recs, state_in, state_out, o, part, a.T, a.H, nC, dir, out_mode, err);
+    gdn::LaunchScope ls(ndir == 2 ? "tc_chain_bidir" : "tc_chain", a.stream);
+    kern<<<dim3(DV / gdn::tc2::kChainNS, a.B * a.H, ndir), gdn::tc2::kChainThreads, SM::kAlloc, a.stream>>>(
+        mk, mq, mo, recs, state_in, state_out, out, a.T, a.H, nC, 0, err);
     return launch_status();
 }
 
 template <int DV, typename Tout>
 gdn_status run_tc(const Args &a, int bidir) {
-    using gdn::tc2::kOutAddPartial;
-    using gdn::tc2::kOutPartial;
-    using gdn::tc2::kOutStore;
     CUtensorMap mk, mq, mv;
     if (!encode_map(&mk, a.k, a.B, a.T, a.H, 128, 64, true) ||
         !encode_map(&mq, a.q, a.B, a.T, a.H, 128, 64, true) ||
@@ -292,18 +301,35 @@ gdn_status run_tc(const Args &a, int bidir) {
     unsigned char *recs = static_cast<unsigned char *>(a.ws);
     gdn_status s = launch_prep<DV>(a, mk, mq, mv, recs, nC, bidir ? 2 : 1, err);
     if (s != GDN_OK) return s;
-    Tout *o = static_cast<Tout *>(a.o);
-    if (!bidir)
-        return launch_chain<DV, Tout>(a, mk, mq, recs, nC, 0, a.state_in, a.state_out, o, nullptr,
-                                      kOutStore, err);
-    // bidirectional: the causal pass writes (o, or an fp32 partial), the reverse pass adds
-    const size_t rec_bytes = round_up(2 * (size_t)a.B * a.H * nC * tc_record_bytes(DV), 256);
-    float *part = std::is_same<Tout, float>::value ? reinterpret_cast<float *>(a.o)
-                                                    : reinterpret_cast<float *>(recs + rec_bytes);
-    const int first = std::is_same<Tout, float>::value ? kOutStore : kOutPartial;
-    s = launch_chain<DV, Tout>(a, mk, mq, recs, nC, 0, nullptr, nullptr, o, part, first, err);
-    if (s != GDN_OK) return s;
-    return launch_chain<DV, Tout>(a, mk, mq, recs, nC, 1, nullptr, nullptr, o, part, kOutAddPartial, err);
+    gdn::tc2::ChainOut<Tout> out{};
+    out.o = static_cast<Tout *>(a.o);
+    if (!bidir) {
+        // the output tile leaves through 128B-swizzled boxes of 128-byte rows
+        constexpr bool f32o = std::is_same<Tout, float>::value;
+        CUtensorMap mo;
+        if (!encode_map(&mo, a.o, a.B, a.T, a.H, DV, f32o ? 32 : 64, true, f32o ? 4 : 2)) return GDN_ERR_CUDA;
+        out.mode = gdn::tc2::kOutStore;
+        return launch_chain<DV, Tout>(a, mk, mq, mo, recs, nC, 1, a.state_in, a.state_out, out, err);
+    }
+    // bidirectional: both directions in one launch; each piece is combined by
+    // whichever of its two producers finishes second
+    constexpr bool f32_out = std::is_same<Tout, float>::value;
+    unsigned char *p = recs + round_up(2 * (size_t)a.B * a.H * nC * tc_record_bytes(DV), 256);
+    const size_t part_bytes = round_up((size_t)a.B * a.T * a.H * DV * sizeof(float), 256);
+    out.mode = gdn::tc2::kOutPair;
+    if (f32_out) {
+        out.part[0] = reinterpret_cast<float *>(a.o);
+    } else {
+        out.part[0] = reinterpret_cast<float *>(p);
+        p += part_bytes;
+    }
+    out.part[1] = reinterpret_cast<float *>(p);
+    p += part_bytes;
+    out.cnt = reinterpret_cast<unsigned int *>(p);
+    if (cudaMemsetAsync(out.cnt, 0, tc_pair_counters(a.B, a.T, a.H, DV) * sizeof(unsigned int), a.stream) !=
+        cudaSuccess)
+        return GDN_ERR_CUDA;
+    return launch_chain<DV, Tout>(a, mk, mq, mq, recs, nC, 2, nullptr, nullptr, out, err);
 }
 
 gdn_status dispatch_tc(const Args &a, int bidir) {

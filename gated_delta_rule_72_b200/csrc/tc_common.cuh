@@ -23,16 +23,25 @@ using namespace gdn::sm100;
 constexpr int kDK = 128;                     // key dimension of the tensor-core path
 constexpr uint32_t kWaitTries = 1u << 24;    // bounded mbarrier polls
 
-// Width of the state slice one chain CTA owns (columns of d_v).
-constexpr int kSliceCols = 32;
+// Width of the U slices in the record (columns of d_v): one chain CTA's slice.
+constexpr int kSliceCols = 64;
+
+// Byte offset of U[row][col] inside one 64 x 64 fp32 slice: 256-byte rows
+// whose 16-byte chunks are XOR-swizzled with row % 8, so that eight threads
+// reading the same columns of eight consecutive rows hit distinct banks.
+__host__ __device__ constexpr int u_off(int row, int col) {
+    return row * 256 + ((((col >> 2) ^ (row & 7)) & 15) << 4) + (col & 3) * 4;
+}
 
 // Per-chunk record written by the prep kernel and read by the chain kernel,
 // rows in FORWARD token order for either direction (the reverse direction's
 // permutation is folded into the record by the prep kernel):
-//   W   bf16, K-major no-swizzle A operand, 64 rows x 128 (d_k)   16384 B
-//   Ph  bf16, K-major no-swizzle A operand, 64 x 64                8192 B
+//   W   bf16, 64 rows x 128 (d_k) as two 128B-swizzled 64-column   16384 B
+//       blocks (the image a SWIZZLE_128B tile load would write), so that
+//       it stacks under the Q tile into one M=128 operand
+//   Ph  bf16, 64 x 64, 128B-swizzled K-major image                  8192 B
 //   Pl  bf16, same layout (P - Ph)                                 8192 B
-//   U   fp32, slice-major [DV/32][64][32] (one slice contiguous)   256*DV B
+//   U   fp32, [DV/64] slices of 64 x 64, rows swizzled (u_off)    256*DV B
 //   dq[64], dkk[64], ds, padding                                   1024 B
 // so that a chain CTA fetches its operands with a handful of bulk copies.
 template <int DV>
@@ -77,6 +86,15 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
     const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
     hi = *reinterpret_cast<const uint32_t *>(&h);
     lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// Element (mn, k) of a 128B-swizzled MN-major operand: 128-byte rows of 64
+// MN elements, one row per k, atoms of 8 rows (1024 B) along k, groups of 64
+// MN elements `mn_group` bytes apart.  (The layout a SWIZZLE_128B tile load
+// writes for a [k][mn] tensor; read with sdesc_sw128_mn.)
+__device__ __forceinline__ int swz_mn(int mn, int k, int mn_group) {
+    return (mn >> 6) * mn_group + (k >> 3) * 1024 + (k & 7) * 128 + ((((mn & 63) >> 3) ^ (k & 7)) << 4) +
+           (mn & 7) * 2;
 }
 
 // Descriptor of a 128B-swizzled operand used MN-major (MN contiguous inside

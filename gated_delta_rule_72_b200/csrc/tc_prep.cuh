@@ -227,7 +227,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     split2(v[2], v[3], hi.y, lo.y);
                     split2(v[4], v[5], hi.z, lo.z);
                     split2(v[6], v[7], hi.w, lo.w);
-                    const int off = kmaj64(fl, f0 + cc * 8);
+                    const int off = sw128(fl, f0 + cc * 8, 0);
                     *reinterpret_cast<uint4 *>(rec + RC::kPh + off) = hi;
                     *reinterpret_cast<uint4 *>(rec + RC::kPl + off) = lo;
                 }
@@ -343,8 +343,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     p1.x = pack_bf16(w[8], w[9]); p1.y = pack_bf16(w[10], w[11]);
                     p1.z = pack_bf16(w[12], w[13]); p1.w = pack_bf16(w[14], w[15]);
                     const int d0 = half * 64 + q * 16;
-                    *reinterpret_cast<uint4 *>(rec + RC::kW + (d0 >> 3) * 1024 + f * 16) = p0;
-                    *reinterpret_cast<uint4 *>(rec + RC::kW + ((d0 + 8) >> 3) * 1024 + f * 16) = p1;
+                    *reinterpret_cast<uint4 *>(rec + RC::kW + sw128(f, d0, 8192)) = p0;
+                    *reinterpret_cast<uint4 *>(rec + RC::kW + sw128(f, d0 + 8, 8192)) = p1;
                 }
             }
 #pragma unroll
@@ -353,13 +353,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 const int col = half * (DV / 2) + q * 16;
                 tmem_ld16(tmem + lane_base + kPrepColU + col, u);
                 tmem_wait_ld();
-                if (row_lane) {   // slice-major: slice col/32, row f, columns col%32 ..
-                    float4 *dst = reinterpret_cast<float4 *>(
-                        rec + RC::kU + (col / kSliceCols) * RC::kUSlice + (f * kSliceCols + col % kSliceCols) * 4);
-                    dst[0] = make_float4(u[0], u[1], u[2], u[3]);
-                    dst[1] = make_float4(u[4], u[5], u[6], u[7]);
-                    dst[2] = make_float4(u[8], u[9], u[10], u[11]);
-                    dst[3] = make_float4(u[12], u[13], u[14], u[15]);
+                if (row_lane) {   // slice col/64, row f, columns col%64 .. +15
+                    unsigned char *sl = rec + RC::kU + (col / kSliceCols) * RC::kUSlice;
+                    const int c0 = col % kSliceCols;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<float4 *>(sl + u_off(f, c0 + 4 * i)) =
+                            make_float4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
                 }
             }
             if (tid < 64) {
