@@ -182,7 +182,7 @@ size_t tc_record_bytes(int dv) {
 // (the causal one is o itself when o is fp32) and one counter per piece.
 size_t tc_pair_counters(int B, int T, int H, int dv) {
     const size_t nC = (size_t)(T + kChunk - 1) / kChunk;
-    return (size_t)B * H * nC * (dv / gdn::tc2::kChainNS) * 8;
+    return (size_t)B * H * nC * (dv / 32);   // one per output tile of the narrowest slices
 }
 
 size_t plan_workspace(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt, int bidir) {
@@ -191,8 +191,8 @@ size_t plan_workspace(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dty
         const size_t nC = (size_t)(T + kChunk - 1) / kChunk;
         size_t bytes = round_up((bidir ? 2 : 1) * (size_t)B * H * nC * tc_record_bytes(dv), 256);
         if (bidir) {
-            const size_t part = round_up((size_t)B * T * H * dv * sizeof(float), 256);
-            bytes += (o_dt == GDN_BF16 ? 2 : 1) * part;
+            // the two directions add up in fp32: in o itself, or (bf16 o) in a buffer
+            if (o_dt == GDN_BF16) bytes += round_up((size_t)B * T * H * dv * sizeof(float), 256);
             bytes += round_up(tc_pair_counters(B, T, H, dv) * sizeof(unsigned int), 256);
         }
         return bytes;
@@ -218,8 +218,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // Tile map over a [B, T, H, d] tensor of bf16 (esize 2) or fp32 (esize 4):
 // boxes of (box_d columns, 1 head, 64 tokens, 1 batch); loads past T read as
-// zero and stores past T are dropped.
-bool encode_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, int box_d, bool swz128,
+// zero and stores past T are dropped.  swz: 0 none, 64 or 128 (bytes).
+bool encode_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, int box_d, int swz,
                 int esize = 2) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) return false;
@@ -228,9 +228,11 @@ bool encode_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, in
     const cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)H * d * es, (cuuint64_t)T * H * d * es};
     const cuuint32_t box[4] = {(cuuint32_t)box_d, 1, 64, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapSwizzle sw = swz == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : swz == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                              : CU_TENSOR_MAP_SWIZZLE_NONE;
     return enc(m, esize == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
-               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               swz128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -274,26 +276,61 @@ gdn_status launch_prep(const Args &a, const CUtensorMap &mk, const CUtensorMap &
     return launch_status();
 }
 
-template <int DV, typename Tout>
+// State columns per chain CTA: 32 while the grid still fits on the SMs (the
+// chain is then latency-bound and the narrower slice halves each step's
+// epilogues), else 64 (half the CTAs and half the record re-reads).
+int chain_slice_cols(int B, int H, int dv, int ndir) {
+    return (long long)B * H * ndir * (dv / 32) <= sm_count() ? 32 : 64;
+}
+
+// o (bf16) <- sum (fp32), n a multiple of 4 elements.
+__global__ void cast_bf16_kernel(const float4 *__restrict__ sum, uint2 *__restrict__ o, size_t n4) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        const float4 v = sum[i];
+        uint2 u;
+        u.x = gdn::tc2::pack_bf16(v.x, v.y);
+        u.y = gdn::tc2::pack_bf16(v.z, v.w);
+        o[i] = u;
+    }
+}
+
+// Output of a chain: target [B, T, H, DV] tensor of Tout (kOutStore) or fp32
+// (kOutPair, both directions adding up there).
+template <int DV, int NS, typename Tout>
 gdn_status launch_chain(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq,
-                        const CUtensorMap &mo, const unsigned char *recs, int nC, int ndir, const float *state_in,
-                        float *state_out, const gdn::tc2::ChainOut<Tout> &out, unsigned int *err) {
-    using SM = gdn::tc2::ChainSmem;
-    auto kern = gdn::tc2::chain_kernel<DV, Tout>;
+                        const unsigned char *recs, int nC, int ndir, const float *state_in,
+                        float *state_out, const gdn::tc2::ChainOut<Tout> &out, const void *target,
+                        unsigned int *err) {
+    using SM = gdn::tc2::ChainSmem<NS>;
+    const bool f32t = std::is_same<Tout, float>::value || out.mode == gdn::tc2::kOutPair;
+    CUtensorMap mo;
+    if (!encode_map(&mo, target, a.B, a.T, a.H, DV, f32t ? 32 : NS, (f32t || NS == 64) ? 128 : 64, f32t ? 4 : 2))
+        return GDN_ERR_CUDA;
+    auto kern = gdn::tc2::chain_kernel<DV, NS, Tout>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
         return GDN_ERR_CUDA;
     gdn::LaunchScope ls(ndir == 2 ? "tc_chain_bidir" : "tc_chain", a.stream);
-    kern<<<dim3(DV / gdn::tc2::kChainNS, a.B * a.H, ndir), gdn::tc2::kChainThreads, SM::kAlloc, a.stream>>>(
+    kern<<<dim3(DV / NS, a.B * a.H, ndir), gdn::tc2::kChainThreads, SM::kAlloc, a.stream>>>(
         mk, mq, mo, recs, state_in, state_out, out, a.T, a.H, nC, 0, err);
     return launch_status();
 }
 
 template <int DV, typename Tout>
+gdn_status launch_chain_ns(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq,
+                           const unsigned char *recs, int nC, int ndir, const float *state_in,
+                           float *state_out, const gdn::tc2::ChainOut<Tout> &out, const void *target,
+                           unsigned int *err) {
+    if (chain_slice_cols(a.B, a.H, DV, ndir) == 32)
+        return launch_chain<DV, 32, Tout>(a, mk, mq, recs, nC, ndir, state_in, state_out, out, target, err);
+    return launch_chain<DV, 64, Tout>(a, mk, mq, recs, nC, ndir, state_in, state_out, out, target, err);
+}
+
+template <int DV, typename Tout>
 gdn_status run_tc(const Args &a, int bidir) {
     CUtensorMap mk, mq, mv;
-    if (!encode_map(&mk, a.k, a.B, a.T, a.H, 128, 64, true) ||
-        !encode_map(&mq, a.q, a.B, a.T, a.H, 128, 64, true) ||
-        !encode_map(&mv, a.v, a.B, a.T, a.H, DV, 64, true))
+    if (!encode_map(&mk, a.k, a.B, a.T, a.H, 128, 64, 128) ||
+        !encode_map(&mq, a.q, a.B, a.T, a.H, 128, 64, 128) ||
+        !encode_map(&mv, a.v, a.B, a.T, a.H, DV, 64, 128))
         return GDN_ERR_CUDA;
     unsigned int *err = timeout_counter();
     if (!err) return GDN_ERR_CUDA;
@@ -302,34 +339,32 @@ gdn_status run_tc(const Args &a, int bidir) {
     gdn_status s = launch_prep<DV>(a, mk, mq, mv, recs, nC, bidir ? 2 : 1, err);
     if (s != GDN_OK) return s;
     gdn::tc2::ChainOut<Tout> out{};
-    out.o = static_cast<Tout *>(a.o);
     if (!bidir) {
-        // the output tile leaves through 128B-swizzled boxes of 128-byte rows
-        constexpr bool f32o = std::is_same<Tout, float>::value;
-        CUtensorMap mo;
-        if (!encode_map(&mo, a.o, a.B, a.T, a.H, DV, f32o ? 32 : 64, true, f32o ? 4 : 2)) return GDN_ERR_CUDA;
         out.mode = gdn::tc2::kOutStore;
-        return launch_chain<DV, Tout>(a, mk, mq, mo, recs, nC, 1, a.state_in, a.state_out, out, err);
+        return launch_chain_ns<DV, Tout>(a, mk, mq, recs, nC, 1, a.state_in, a.state_out, out, a.o, err);
     }
-    // bidirectional: both directions in one launch; each piece is combined by
-    // whichever of its two producers finishes second
+    // bidirectional: both directions in one launch, adding up in fp32 (in o
+    // itself for an fp32 o, else in a buffer that is then rounded into o)
     constexpr bool f32_out = std::is_same<Tout, float>::value;
     unsigned char *p = recs + round_up(2 * (size_t)a.B * a.H * nC * tc_record_bytes(DV), 256);
-    const size_t part_bytes = round_up((size_t)a.B * a.T * a.H * DV * sizeof(float), 256);
-    out.mode = gdn::tc2::kOutPair;
-    if (f32_out) {
-        out.part[0] = reinterpret_cast<float *>(a.o);
-    } else {
-        out.part[0] = reinterpret_cast<float *>(p);
-        p += part_bytes;
+    const size_t n = (size_t)a.B * a.T * a.H * DV;
+    void *target = a.o;
+    if (!f32_out) {
+        target = p;
+        p += round_up(n * sizeof(float), 256);
     }
-    out.part[1] = reinterpret_cast<float *>(p);
-    p += part_bytes;
+    out.mode = gdn::tc2::kOutPair;
     out.cnt = reinterpret_cast<unsigned int *>(p);
     if (cudaMemsetAsync(out.cnt, 0, tc_pair_counters(a.B, a.T, a.H, DV) * sizeof(unsigned int), a.stream) !=
         cudaSuccess)
         return GDN_ERR_CUDA;
-    return launch_chain<DV, Tout>(a, mk, mq, mq, recs, nC, 2, nullptr, nullptr, out, err);
+    s = launch_chain_ns<DV, Tout>(a, mk, mq, recs, nC, 2, nullptr, nullptr, out, target, err);
+    if (s != GDN_OK || f32_out) return s;
+    gdn::LaunchScope ls("tc_bidir_cast", a.stream);
+    const size_t n4 = n / 4;
+    const int grid = (int)((n4 + 255) / 256 < (size_t)sm_count() * 8 ? (n4 + 255) / 256 : (size_t)sm_count() * 8);
+    cast_bf16_kernel<<<grid, 256, 0, a.stream>>>(static_cast<const float4 *>(target), static_cast<uint2 *>(a.o), n4);
+    return launch_status();
 }
 
 gdn_status dispatch_tc(const Args &a, int bidir) {

@@ -1,39 +1,49 @@
 // tc_chain.cuh -- the inter-chunk state chain on the tensor cores.
 //
-// One CTA owns one (b, h), one direction and a slice of NS = 64 columns of
-// the d_k x d_v state (the columns evolve independently).  It walks the
+// One CTA owns one (b, h), one direction and a slice of NS columns (32 or 64)
+// of the d_k x d_v state (the columns evolve independently).  It walks the
 // chunks in order (the reverse direction from the last chunk to the first)
 // keeping its state slice on chip: an fp32 master copy in registers and a
 // bf16 hi/lo copy in shared memory as the B operand of the tensor-core
 // products.  Per chunk, from the prep record (rows in forward token order)
 // and the bf16 Q and K tiles:
 //   [Y; X] = [Q; W] [S_hi | S_lo]            one M=128 product
-//   Delta = U - X
-//   S <- ds S + K^T [E_hi | E_lo],  E = diag(dkk) Delta
+//   Delta = U - X,  E = diag(dkk) Delta
+//   S <- ds S + K^T [E_hi | E_lo]
 //   O = diag(dq) Y + [P_hi | P_lo] [D; D],  D = [Delta_hi | Delta_lo]
 // The hi and lo halves of a split operand sit side by side along N, so one
 // MMA of width 2*NS yields both partial products; P's halves are stacked
 // along K instead, so the tensor core adds P_hi D + P_lo D itself.  Stacking
-// Q over W makes Y and X one instruction stream (a tcgen05.mma costs its
-// issuing thread tens of cycles whatever its size, so fewer, wider products
-// are faster); Y then lands in TMEM lanes 0-63 and X in lanes 64-127.
+// Q over W makes Y and X one instruction stream; Y then lands in TMEM lanes
+// 0-63 and X in lanes 64-127.
 //
-// Roles (20 warps).  The 16 epilogue warps cover the 128 TMEM lanes four
-// times (warp w reads lane quarter w % 4, columns 16 * (w / 4) .. +15):
-//   quarters 2, 3 (X rows)  form Delta and E           (critical path)
-//   quarters 0, 1 (Y rows)  form and store the output   (off the chain)
+// What bounds a step.  An MMA stream (one issuing thread, one accumulator)
+// completes one K=16 instruction per ~130 cycles whatever N is, so each
+// product is split over two streams where TMEM has room.  The epilogues are
+// bound by instruction issue (splitting a value into bf16 hi/lo costs about
+// three instructions), and a TMEM lane quarter can only be read by the warps
+// of the matching SM sub-partition, so the X rows' epilogue runs on two of
+// the four.  NS = 32 halves the epilogues at the same MMA count; NS = 64
+// halves the CTAs (and the record traffic) for a given head count.
+//
+// Roles (21 warps).  The 16 epilogue warps cover the 128 TMEM lanes four
+// times (warp w reads lane quarter w % 4, columns NS/4 * (w / 4) .. +NS/4-1):
+//   quarters 2, 3 (X rows)  form Delta, D and E        (critical path)
+//   quarters 0, 1 (Y rows)  form and stage the output   (off the chain)
 //   all                     S <- ds S + K^T E, thread = one row of S
-// Warps 16 and 17 issue [Q;W] S, one K half each (A then also K^T E), warp 19
-// issues P D and warp 18 loads the stages.  A thread that has just queued a
-// batch of MMAs is slow to see barriers complete, so the off-chain product
-// gets an issuing thread of its own.
-// The roles meet on mbarriers; each of them can only complete its next phase
+// Warps 16 and 17 issue [Q;W] S, one K half each, and K^T E (one token half
+// each when TMEM holds two accumulators for it, else warp 16 alone); warp 19
+// issues P D, warp 20 stores the output tiles and warp 18 loads the stages.  The
+// roles meet on mbarriers, each of which can only complete its next phase
 // after every waiter has observed the previous one.
 //
-// Bidirectional mode runs both directions in one launch (grid.z = 2).  Each
-// direction writes its 32 x 16 output pieces to its own fp32 buffer; of the
-// two CTAs that produce the same piece, the one that finishes second (an
-// atomic counter per piece decides) adds the other's piece and writes o.
+// Bidirectional mode runs both directions in one launch (grid.z = 2), and
+// both write the same fp32 output tiles.  An atomic counter per tile decides
+// the order: the first of the two CTAs TMA-stores its tile and then marks it
+// landed; the second waits for that mark (the two directions reach a given
+// tile at very different times, so it seldom waits) and TMA-reduce-adds its
+// own tile onto it.  The first one's mark does not depend on any other CTA,
+// and the second only waits on a CTA that is already running.
 #pragma once
 
 #include "tc_common.cuh"
@@ -45,44 +55,46 @@ namespace tc2 {
 // Development aid (not built into the library): cycle stamps of CTA (0,0,0),
 // steps 10..19.
 __device__ long long g_chain_ts[10][32];
+__device__ long long g_chain_rarr[10][20];   // per-warp arrival on the S-rewritten barrier
 #define CHAIN_TS(slot) do { if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && \
     step >= 10 && step < 20) g_chain_ts[step - 10][slot] = clock64(); } while (0)
 #else
 #define CHAIN_TS(slot) do { } while (0)
 #endif
 
-constexpr int kChainNS = 64;           // state columns per CTA
-
+template <int NS>
 struct ChainSmem {
-    static constexpr int NS = kChainNS;
-    // one stage (1024-aligned): [Q;W] 2 x 16 KB column blocks (Q rows 0-63,
+    static_assert(NS == 32 || NS == 64, "slice width");
+    // One stage (1024-aligned): [Q;W] 2 x 16 KB column blocks (Q rows 0-63,
     // W rows 64-127), K 2 x 8 KB, P_hi | P_lo 2 x 8 KB (all 128B-swizzled,
-    // K-major), U 64 x 64 fp32 (rows swizzled, u_off).  The operands the epilogues write,
-    // [S_hi | S_lo], [D_hi | D_lo] and [E_hi | E_lo], are 128B-swizzled
-    // MN-major (one 128-byte row per K index), like a tile load would write
-    // them: the unswizzled layouts cost the tensor core several times the
-    // shared-memory wavefronts.
+    // K-major), U as NS/32 granules of 64 x 32 fp32 (rows swizzled, u_off).
+    // The operands the epilogues write, [S_hi | S_lo], [D_hi | D_lo] and
+    // [E_hi | E_lo], are 128B-swizzled MN-major (one 128-byte row of 64 MN
+    // elements per K index, hi and lo halves in separate 64-element groups when
+    // NS = 64), as a tile load would write them: unswizzled layouts cost the
+    // tensor core several times the shared-memory wavefronts.
     static constexpr int kQW = 0;
     static constexpr int kK = 32768;
     static constexpr int kP = kK + 16384;
     static constexpr int kU = kP + 16384;
     static constexpr int kStage = kU + 64 * NS * 4;
-    static constexpr int kSL = 2 * kStage;                 // [S_hi | S_lo], K = 128: 2 x 16 KB
-    static constexpr int kD = kSL + 128 * 2 * NS * 2;      // [D_hi | D_lo], K = 64: 2 x 8 KB
-    static constexpr int kE = kD + 64 * 2 * NS * 2;        // [E_hi | E_lo]
+    static constexpr int kSL = 2 * kStage;                 // [S_hi | S_lo], K = 128
+    static constexpr int kD = kSL + 128 * 2 * NS * 2;      // [D_hi | D_lo], K = 64
+    static constexpr int kE = kD + 64 * 2 * NS * 2;        // [E_hi | E_lo], K = 64
     static constexpr int kG = kE + 64 * 2 * NS * 2;        // 2 x gates (dq, dkk, ds)
     static constexpr int kGate = 528;
     static constexpr int kBar = kG + 2 * kGate;            // mbarriers
     static constexpr int kCtl = kBar + 128;
     static constexpr int kBytes = kCtl + 16;
     static constexpr int kAlloc = kBytes + 1024;
+    // MN-group strides of the swizzled B operands (used when 2 * NS > 64)
+    static constexpr int kGrpSL = 128 * 128, kGrpDE = 64 * 128;
     static_assert(kStage % 1024 == 0 && kSL % 1024 == 0 && kD % 1024 == 0 && kE % 1024 == 0,
                   "swizzled operands must stay 1024-aligned");
-    static_assert(NS == 64, "one 64-element MN group per hi / lo half");
     static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
-constexpr int kChainWarps = 20;
+constexpr int kChainWarps = 21;
 constexpr int kChainThreads = kChainWarps * 32;
 
 enum OutMode { kOutStore = 0, kOutPair = 1 };
@@ -99,42 +111,68 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, float4 v
     *reinterpret_cast<uint2 *>(p) = u;
 }
 
-// Output of a chain: where each direction's pieces go and how they combine.
+// Output of a chain.  kOutStore: tm_o maps o ([B, T, H, DV], Tout).  kOutPair
+// (both directions): tm_o maps an fp32 [B, T, H, DV] sum (o itself when Tout
+// is float), cnt holds one counter per output tile, zero on entry.
 template <typename Tout>
 struct ChainOut {
-    Tout *o;                 // [B, T, H, DV]
-    float *part[2];          // kOutPair: fp32 [B, T, H, DV] per direction (part[0] may be o)
-    unsigned int *cnt;       // kOutPair: one counter per 32 x 16 piece, zero on entry
+    unsigned int *cnt;
     int mode;
 };
 
+// Staging of one output tile (64 rows x NS columns) for its TMA store: byte
+// offset of the 16-byte chunk that starts at column `col` of row `row`.
+// fp32: boxes of 32 columns (128-byte rows, 8 KB each, 128B swizzle); bf16:
+// one box of NS columns (128B swizzle for 128-byte rows, 64B for 64-byte rows).
+template <int NS, typename Tout>
+__device__ __forceinline__ int out_stage_off(int row, int col) {
+    if (sizeof(Tout) == 4) return (col >> 5) * 8192 + swz128(row * 128 + (col & 31) * 4);
+    return NS == 64 ? swz128(row * 128 + col * 2) : swz64(row * 64 + col * 2);
+}
+
+// NC consecutive TMEM columns (8 or 16) of this warp's lane quarter.
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float *v) {
+    if (NC == 16) {
+        tmem_ld16(taddr, v);
+    } else {
+        uint32_t r[8];
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                       "=r"(r[6]), "=r"(r[7])
+                     : "r"(taddr));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+    }
+}
+
 // grid (DV/NS, B*H, directions), block kChainThreads.  blockIdx.z + dir0 is
 // the direction (0 causal, 1 reverse).
-template <int DV, typename Tout>
+template <int DV, int NS, typename Tout>
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-             const __grid_constant__ CUtensorMap tm_o, const unsigned char *__restrict__ recs, const float *__restrict__ state_in,
-             float *__restrict__ state_out, const ChainOut<Tout> out, int T, int H, int nC,
-             int dir0, unsigned int *__restrict__ err)
+             const __grid_constant__ CUtensorMap tm_o, const unsigned char *__restrict__ recs,
+             const float *__restrict__ state_in, float *__restrict__ state_out, const ChainOut<Tout> out,
+             int T, int H, int nC, int dir0, unsigned int *__restrict__ err)
 {
-    using SM = ChainSmem;
+    using SM = ChainSmem<NS>;
     using RC = Rec<DV>;
-    constexpr int NS = kChainNS;
-    constexpr int N2 = 2 * NS;
+    constexpr int N2 = 2 * NS;          // accumulator width: hi | lo
+    constexpr int NC = NS / 4;          // columns per epilogue warp
+    constexpr bool kSplitS = 5 * N2 <= 512;   // K^T E in two streams (own TMEM columns)
     extern __shared__ __align__(16) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kBar);
-    uint64_t *full = bars + 0;         // [2] stage loaded                        (loader -> all)
-    uint64_t *free_st = bars + 2;      // [2] stage consumed: 16 warps, A, B, C x 2  (-> loader)
-    uint64_t *xy_bar = bars + 4;       // [Y; X] complete, 2 commits              (A, B -> warps)
-    uint64_t *delta_bar = bars + 5;    // Delta (fp32) in the stage, 8 X warps    (-> Y warps)
-    uint64_t *e_bar = bars + 6;        // E written (and Y read), 8 Y warps       (-> A, B)
-    uint64_t *dd_bar = bars + 7;       // D written, 8 X warps                    (-> C)
-    uint64_t *s_bar = bars + 8;        // K^T E complete, 2 commits               (A, B -> warps, C)
-    uint64_t *r_bar = bars + 9;        // S rewritten, 16 warps                   (-> A, B)
-    uint64_t *pd_bar = bars + 10;      // P D complete                            (C -> warps)
-    uint64_t *pd_free = bars + 11;     // P D read, 8 Y warps                     (-> C)
-    uint64_t *o_bar = bars + 12;       // output tile staged, 8 Y warps           (-> C)
+    uint64_t *full = bars + 0;         // [2] stage loaded                          (loader -> all)
+    uint64_t *free_st = bars + 2;      // [2] stage consumed: 16 warps, A, B, C, storer (-> loader)
+    uint64_t *xy_bar = bars + 4;       // [Y; X] complete, 2 commits                (A, B -> warps)
+    uint64_t *d_bar = bars + 5;        // D and E written, 8 X warps                (-> A, B, C)
+    uint64_t *s_bar = bars + 6;        // K^T E complete, 1 or 2 commits            (-> warps, C)
+    uint64_t *r_bar = bars + 7;        // S rewritten, 16 warps                     (-> A, B)
+    uint64_t *pd_bar = bars + 8;       // P D complete                              (C -> warps)
+    uint64_t *pd_free = bars + 9;      // P D read, 8 Y warps                       (-> C)
+    uint64_t *o_bar = bars + 10;       // output tile staged, 8 Y warps             (-> storer)
+    uint64_t *o_seen = bars + 11;      // storer has seen o_bar's phase             (-> Y warps)
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + SM::kCtl);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + SM::kCtl + 4);
 
@@ -146,13 +184,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     const int nbh = gridDim.y;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const int n0 = cg * 16;                                 // this warp's 16 columns of the slice
-    // TMEM columns, each accumulator 2*NS wide (hi | lo): [Y;X] in two K halves
-    // (XA, XB), K^T E in two token halves (S, and XB again once [Y;X] is read), P D
-    constexpr uint32_t kColXA = 0, kColXB = N2, kColS = 2 * N2, kColPD = 3 * N2;
+    const int n0 = cg * NC;                                 // this warp's columns of the slice
+    // TMEM columns, each accumulator 2*NS wide (hi | lo): [Y;X] in two K halves,
+    // K^T E (two token halves when kSplitS), P D
+    constexpr uint32_t kColXA = 0, kColXB = N2, kColS = 2 * N2, kColPD = 3 * N2, kColSB = 4 * N2;
     constexpr uint32_t kCols = 512;
     static_assert(4 * N2 <= 512, "TMEM budget");
-    static_assert(NS == kSliceCols, "the record stores U in slices of the chain's width");
+    static_assert(NS % kSliceCols == 0, "the record stores U in granules of kSliceCols columns");
     const unsigned char *rec_base = recs + (size_t)(dir * nbh + bh) * nC * RC::kBytes;
 
     if (tid == 0) {
@@ -161,38 +199,40 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         mbar_init(&free_st[0], 20);
         mbar_init(&free_st[1], 20);
         mbar_init(xy_bar, 2);
-        mbar_init(delta_bar, 8);
-        mbar_init(e_bar, 8);
-        mbar_init(dd_bar, 8);
-        mbar_init(s_bar, 2);
+        mbar_init(d_bar, 8);
+        mbar_init(s_bar, kSplitS ? 2 : 1);
         mbar_init(r_bar, 16);
         mbar_init(pd_bar, 1);
         mbar_init(pd_free, 8);
         mbar_init(o_bar, 8);
+        mbar_init(o_seen, 1);
         fence_mbar_init();
         *abort_s = 0;
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_q);
-        if (out.mode == kOutStore) prefetch_tensormap(&tm_o);
+        prefetch_tensormap(&tm_o);
     }
     if (warp == 0) {
         tmem_alloc(tmem_base_s, kCols);
         tmem_relinquish();
     }
-    // state: epilogue thread (quarter, cg, lane) owns row d_row, columns n0 .. n0+15
+    // Offsets of this thread's pieces of the split operands.  State: epilogue
+    // thread (quarter, cg, lane) owns row d_row, columns n0 .. n0+NC-1.
     const int d_row = quarter * 32 + lane;
-    float S[16];
+    auto sl_off = [&](int n, int k) { return (N2 > 64 ? (n >> 6) * SM::kGrpSL : 0) + swz128(k * 128 + (n & 63) * 2); };
+    auto de_off = [&](int n, int k) { return (N2 > 64 ? (n >> 6) * SM::kGrpDE : 0) + swz128(k * 128 + (n & 63) * 2); };
+    float S[NC];
     if (warp < 16) {
         const float *src = state_in ? state_in + ((size_t)bh * kDK + d_row) * DV + j0 + n0 : nullptr;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) S[n] = src ? src[n] : 0.f;
+        for (int n = 0; n < NC; ++n) S[n] = src ? src[n] : 0.f;
 #pragma unroll
-        for (int n = 0; n < 16; n += 8) {
+        for (int n = 0; n < NC; n += 8) {
             uint4 hi, lo;
             split2(S[n], S[n + 1], hi.x, lo.x); split2(S[n + 2], S[n + 3], hi.y, lo.y);
             split2(S[n + 4], S[n + 5], hi.z, lo.z); split2(S[n + 6], S[n + 7], hi.w, lo.w);
-            *reinterpret_cast<uint4 *>(smem + SM::kSL + swz_mn(n0 + n, d_row, 16384)) = hi;
-            *reinterpret_cast<uint4 *>(smem + SM::kSL + swz_mn(NS + n0 + n, d_row, 16384)) = lo;
+            *reinterpret_cast<uint4 *>(smem + SM::kSL + sl_off(n0 + n, d_row)) = hi;
+            *reinterpret_cast<uint4 *>(smem + SM::kSL + sl_off(NS + n0 + n, d_row)) = lo;
         }
     }
     fence_async_shared();
@@ -208,16 +248,22 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             if (err) atomicAdd(err, 1u);
         }
     };
+    // issuing threads spin instead (a suspended try_wait can oversleep the phase)
+    auto spin_on = [&](uint64_t *bar, uint32_t parity) {
+        if (!mbar_spin(bar, parity, kSpinTries)) {
+            *abort_s = 1;
+            if (err) atomicAdd(err, 1u);
+        }
+    };
     auto stage_addr = [&](int step) { return sbase + (step & 1) * SM::kStage; };
     auto gates = [&](int step) { return reinterpret_cast<const float *>(smem + SM::kG + (step & 1) * SM::kGate); };
     auto adv = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
     constexpr uint32_t idQW = idesc(128, N2, 1, 0, 1);   // [Q;W] S and P D: A K-major, B MN-major
     constexpr uint32_t idKE = idesc(128, N2, 1, 1, 1);   // K^T E: A MN-major (the K tile), B MN-major
-    const uint64_t dK0 = sdesc_sw128_mn(sbase + SM::kK, 8192);
     // MN-major swizzled B operands; a K-step of 16 rows advances 2048 bytes
-    const uint64_t dSL = sdesc_sw128_mn(sbase + SM::kSL, 16384);
-    const uint64_t dD = sdesc_sw128_mn(sbase + SM::kD, 8192);
-    const uint64_t dE = sdesc_sw128_mn(sbase + SM::kE, 8192);
+    const uint64_t dSL = sdesc_sw128_mn(sbase + SM::kSL, SM::kGrpSL);
+    const uint64_t dD = sdesc_sw128_mn(sbase + SM::kD, SM::kGrpDE);
+    const uint64_t dE = sdesc_sw128_mn(sbase + SM::kE, SM::kGrpDE);
 
     if (warp == 18) {
         // ============================ loader ========================================
@@ -229,7 +275,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     wait_on(&free_st[buf], (free_phases >> buf) & 1u);
                     free_phases ^= 1u << buf;
                 }
-                CHAIN_TS(24);
                 if (*abort_s) break;
                 const int c = chunk_of(step);
                 unsigned char *st = smem + buf * SM::kStage;
@@ -244,26 +289,27 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 tma_load_4d(st + SM::kK, &tm_k, bar, 0, h, t0, b);
                 tma_load_4d(st + SM::kK + 8192, &tm_k, bar, 64, h, t0, b);
                 bulk_load(st + SM::kP, rec + RC::kPh, 16384, bar);
-                bulk_load(st + SM::kU, rec + RC::kU + slice * RC::kUSlice, RC::kUSlice, bar);
+                bulk_load(st + SM::kU, rec + RC::kU + j0 * 64 * 4, 64 * NS * 4, bar);
                 bulk_load(smem + SM::kG + buf * SM::kGate, rec + RC::kGate, SM::kGate, bar);
             }
         }
         __syncwarp();
     } else if (warp == 16 || warp == 17) {
         // ===== issuers A (warp 16) and B (warp 17): half of [Q;W] S each (d_k 0-63 /
-        // 64-127), then half of K^T E each (tokens 0-31 / 32-63; B accumulates into
-        // its [Y;X] columns, which every reader has drained by the time E is ready)
+        // 64-127), then K^T E: tokens 0-31 / 32-63 into separate accumulators
+        // when kSplitS, else all of it from A
         if (lane == 0) {
             const int part = warp - 16;
             const uint32_t colXY = part ? kColXB : kColXA;
-            const uint32_t colS = part ? kColXB : kColS;
-            uint32_t full_phases = 0, e_phase = 0, r_phase = 0;
+            const uint32_t colS = part ? kColSB : kColS;
+            uint32_t full_phases = 0, d_phase = 0, r_phase = 0;
             for (int step = 0; step < nC; ++step) {
                 const int buf = step & 1;
                 const uint32_t st = stage_addr(step);
                 if (part == 0) CHAIN_TS(0);
                 wait_on(&full[buf], (full_phases >> buf) & 1u);
                 full_phases ^= 1u << buf;
+                if (part == 0) CHAIN_TS(25);
                 if (step > 0) { wait_on(r_bar, r_phase); r_phase ^= 1; }
                 if (part == 0) CHAIN_TS(1); else CHAIN_TS(23);
                 if (*abort_s) break;
@@ -278,37 +324,38 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 #ifdef GDN_CHAIN_TIMING
                 if (part == 0) { mbar_wait(xy_bar, step & 1, kWaitTries); CHAIN_TS(7); }
 #endif
-                wait_on(e_bar, e_phase);
-                e_phase ^= 1;
-                if (part == 0) CHAIN_TS(2);
-                if (*abort_s) break;
-                tc_fence_after();
-                const uint64_t dK = sdesc_sw128_mn(st + SM::kK, 8192);   // this stage's K tile
+                if (kSplitS || part == 0) {
+                    wait_on(d_bar, d_phase);
+                    d_phase ^= 1;
+                    if (part == 0) CHAIN_TS(2);
+                    if (*abort_s) break;
+                    tc_fence_after();
+                    const uint64_t dK = sdesc_sw128_mn(st + SM::kK, 8192);   // this stage's K tile
+                    constexpr int kSteps = kSplitS ? 2 : 4;
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const int s = part * 2 + k;
-                    mma_bf16(tmem + colS, adv(dK, s * 2048), adv(dE, s * 2048), idKE, k > 0);
+                    for (int k = 0; k < kSteps; ++k) {
+                        const int s = part * kSteps + k;
+                        mma_bf16(tmem + colS, adv(dK, s * 2048), adv(dE, s * 2048), idKE, k > 0);
+                    }
+                    mma_commit(s_bar);
+                    if (part == 0) CHAIN_TS(3);
                 }
-                mma_commit(s_bar);
-                if (part == 0) CHAIN_TS(3);
                 mma_commit(&free_st[buf]);
             }
         }
         __syncwarp();
     } else if (warp == 19) {
         // ===== issuer C: P D once D is written and K^T E is done (the chain's
-        // product goes first) and the output warps have drained the previous P D;
-        // then the TMA store of the staged output tile
+        // product goes first) and the output warps have drained the previous P D
         if (lane == 0) {
-            uint32_t full_phases = 0, dd_phase = 0, s_phase = 0, pf_phase = 0, o_phase = 0;
+            uint32_t full_phases = 0, d_phase = 0, s_phase = 0, pf_phase = 0;
             for (int step = 0; step < nC; ++step) {
                 const int buf = step & 1;
-                const int c = chunk_of(step);
                 const uint32_t st = stage_addr(step);
                 wait_on(&full[buf], (full_phases >> buf) & 1u);
                 full_phases ^= 1u << buf;
-                wait_on(dd_bar, dd_phase);
-                dd_phase ^= 1;
+                wait_on(d_bar, d_phase);
+                d_phase ^= 1;
                 wait_on(s_bar, s_phase);
                 s_phase ^= 1;
                 CHAIN_TS(4);
@@ -326,51 +373,68 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 mma_commit(pd_bar);
                 CHAIN_TS(5);
                 mma_commit(&free_st[buf]);
-                if (out.mode == kOutStore) {
-                    // the output warps staged the tile in this stage's U region
-                    wait_on(o_bar, o_phase);
-                    o_phase ^= 1;
-                    if (*abort_s) break;
-                    const unsigned char *ob = smem + buf * SM::kStage + SM::kU;
-                    if (sizeof(Tout) == 4) {
-                        tma_store_4d(&tm_o, ob, j0, h, c * 64, b);
-                        tma_store_4d(&tm_o, ob + 8192, j0 + 32, h, c * 64, b);
-                    } else {
-                        tma_store_4d(&tm_o, ob, j0, h, c * 64, b);
-                    }
-                    bulk_commit_group();
-                    bulk_wait_read_all();   // the stage may be reloaded after this
-                    CHAIN_TS(24);
-                }
-                mbar_arrive(&free_st[buf]);
             }
-            if (out.mode == kOutStore) bulk_wait_all();   // the output stores have landed
+        }
+        __syncwarp();
+    } else if (warp == 20) {
+        // ===== storer: the staged output tile leaves by TMA; in a bidirectional
+        // scan the second of the two directions adds its tile onto the first's
+        if (lane == 0) {
+            uint32_t o_phase = 0;
+            for (int step = 0; step < nC; ++step) {
+                const int buf = step & 1;
+                const int c = chunk_of(step);
+                // the output warps staged the tile over this stage's U region
+                wait_on(o_bar, o_phase);
+                o_phase ^= 1;
+                mbar_arrive(o_seen);   // o_bar may complete its next phase
+                if (*abort_s) break;
+                const unsigned char *ob = smem + buf * SM::kStage + SM::kU;
+                bool add = false;      // TMA-reduce-add onto the other direction's tile
+                size_t tile = 0;
+                if (out.mode == kOutPair) {
+                    tile = ((size_t)bh * nC + c) * gridDim.x + slice;
+                    if (atomicAdd(out.cnt + tile, 1u) != 0u) {
+                        // second: wait for the first one's "landed" mark (+2)
+                        uint32_t n = 0;
+                        while (ld_acquire_gpu(out.cnt + tile) < 3u && ++n < kSpinTries) {}
+                        if (n >= kSpinTries) {
+                            *abort_s = 1;
+                            if (err) atomicAdd(err, 1u);
+                            break;
+                        }
+                        fence_proxy_async_global();
+                        add = true;
+                    }
+                }
+                if (sizeof(Tout) == 4 || out.mode == kOutPair) {
+#pragma unroll
+                    for (int x = 0; x < NS / 32; ++x) {
+                        if (add) tma_reduce_add_4d(&tm_o, ob + x * 8192, j0 + 32 * x, h, c * 64, b);
+                        else tma_store_4d(&tm_o, ob + x * 8192, j0 + 32 * x, h, c * 64, b);
+                    }
+                } else {
+                    tma_store_4d(&tm_o, ob, j0, h, c * 64, b);
+                }
+                bulk_commit_group();
+                bulk_wait_read_all();            // the stage may be reloaded after this
+                CHAIN_TS(27);
+                mbar_arrive(&free_st[buf]);
+                if (out.mode == kOutPair && !add) {
+                    bulk_wait_all();             // landed in global memory: mark it (+2)
+                    fence_proxy_async_global();
+                    __threadfence();
+                    atomicAdd(out.cnt + tile, 2u);
+                }
+            }
+            bulk_wait_all();   // the output stores have landed
         }
         __syncwarp();
     } else {
         // ============================ epilogue warps (0..15) ========================
-        // Lane quarter 2, 3 warps (X rows) and quarter 0, 1 warps (Y rows) pair up:
-        // X warp (q + 2, cg) and Y warp (q, cg) cover the same 32 token rows and 16
-        // columns.  X forms Delta (into the stage's U region, in place) and D; Y
-        // forms E from that Delta, so both halves of the lane-quarter <-> SM
-        // sub-partition binding share the Delta epilogue.
         const bool xrows = quarter >= 2;                 // TMEM lanes 64-127 hold X
         const int r = xrows ? d_row - 64 : d_row;        // token row (forward order) of this lane
-        int uo[4], so[4], oo[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uo[q] = u_off(r, n0 + 4 * q);
-            // output staging: fp32 boxes of 32 columns, or one bf16 box of 64
-            oo[q] = sizeof(Tout) == 4 ? ((n0 + 4 * q) >> 5) * 8192 + sw128(r, ((n0 + 4 * q) & 31) * 2, 0)
-                                      : sw128(r, n0 + 4 * q, 0);   // q = 0, 2 used
-        }
-        const int dof[4] = {swz_mn(n0, r, 8192), swz_mn(n0 + 8, r, 8192), swz_mn(NS + n0, r, 8192),
-                            swz_mn(NS + n0 + 8, r, 8192)};
-        so[0] = swz_mn(n0, d_row, 16384);
-        so[1] = swz_mn(n0 + 8, d_row, 16384);
-        so[2] = swz_mn(NS + n0, d_row, 16384);
-        so[3] = swz_mn(NS + n0 + 8, d_row, 16384);
-        uint32_t full_phases = 0, xy_phase = 0, dl_phase = 0, s_phase = 0, pd_phase = 0;
+        uint32_t full_phases = 0, xy_phase = 0, s_phase = 0, pd_phase = 0, os_phase = 0;
         for (int step = 0; step < nC; ++step) {
             const int buf = step & 1;
             const int c = chunk_of(step);
@@ -381,83 +445,62 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             if (tid == 0) CHAIN_TS(14);
             const float *gt = gates(step);
             const float ds = gt[128];
-            const float dq = gt[r], dkk = gt[64 + r];
+            const float dg = xrows ? gt[64 + r] : gt[r];   // dkk for X rows, dq for Y rows
             // X rows overwrite D below: the previous P D must have read it
             if (xrows && step > 0) { wait_on(pd_bar, pd_phase); pd_phase ^= 1; }
             wait_on(xy_bar, xy_phase);
             xy_phase ^= 1;
             if (*abort_s) break;
             tc_fence_after();
-            float acc[16];   // X (or Y) = (A hi + A lo) + (B hi + B lo)
+            float acc[NC];   // X (or Y) = (A hi + A lo) + (B hi + B lo)
             {
-                float a0[16], a1[16], a2[16], a3[16];
-                tmem_ld16(tmem + lane_base + kColXA + n0, a0);
-                tmem_ld16(tmem + lane_base + kColXA + NS + n0, a1);
-                tmem_ld16(tmem + lane_base + kColXB + n0, a2);
-                tmem_ld16(tmem + lane_base + kColXB + NS + n0, a3);
+                float a0[NC], a1[NC], a2[NC], a3[NC];
+                tmem_ld_cols<NC>(tmem + lane_base + kColXA + n0, a0);
+                tmem_ld_cols<NC>(tmem + lane_base + kColXA + NS + n0, a1);
+                tmem_ld_cols<NC>(tmem + lane_base + kColXB + n0, a2);
+                tmem_ld_cols<NC>(tmem + lane_base + kColXB + NS + n0, a3);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) acc[e] = (a0[e] + a1[e]) + (a2[e] + a3[e]);
+                for (int e = 0; e < NC; ++e) acc[e] = (a0[e] + a1[e]) + (a2[e] + a3[e]);
             }
-            tc_fence_before();
             if (tid == 0) CHAIN_TS(15);
             if (xrows) {
                 if (tid == 64) CHAIN_TS(10);
-                // Delta = U - X, written back over U for the Y warps
-                float d[16];
+                float d[NC];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float4 u = *reinterpret_cast<const float4 *>(ureg + uo[q]);
-                    u.x -= acc[4 * q]; u.y -= acc[4 * q + 1]; u.z -= acc[4 * q + 2]; u.w -= acc[4 * q + 3];
-                    *reinterpret_cast<float4 *>(ureg + uo[q]) = u;
-                    d[4 * q] = u.x; d[4 * q + 1] = u.y; d[4 * q + 2] = u.z; d[4 * q + 3] = u.w;
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(delta_bar);
-                    mbar_arrive(&free_st[buf]);   // done with the stage (Y warps hold it)
+                for (int q = 0; q < NC / 4; ++q) {
+                    const int col = n0 + 4 * q;
+                    const float4 u = *reinterpret_cast<const float4 *>(ureg + (col >> 5) * RC::kUSlice + u_off(r, col & 31));
+                    d[4 * q] = u.x - acc[4 * q];
+                    d[4 * q + 1] = u.y - acc[4 * q + 1];
+                    d[4 * q + 2] = u.z - acc[4 * q + 2];
+                    d[4 * q + 3] = u.w - acc[4 * q + 3];
                 }
                 if (tid == 64) CHAIN_TS(21);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&free_st[buf]);   // done reading the stage
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const float *x = d + 8 * hh;
-                    uint4 dh, dl;
+                for (int h8 = 0; h8 < NC; h8 += 8) {
+                    const float *x = d + h8;
+                    uint4 dh, dl, eh, el;
                     split2(x[0], x[1], dh.x, dl.x); split2(x[2], x[3], dh.y, dl.y);
                     split2(x[4], x[5], dh.z, dl.z); split2(x[6], x[7], dh.w, dl.w);
-                    *reinterpret_cast<uint4 *>(smem + SM::kD + dof[hh]) = dh;
-                    *reinterpret_cast<uint4 *>(smem + SM::kD + dof[2 + hh]) = dl;
+                    split2(dg * x[0], dg * x[1], eh.x, el.x); split2(dg * x[2], dg * x[3], eh.y, el.y);
+                    split2(dg * x[4], dg * x[5], eh.z, el.z); split2(dg * x[6], dg * x[7], eh.w, el.w);
+                    const int oh = de_off(n0 + h8, r), ol = de_off(NS + n0 + h8, r);
+                    *reinterpret_cast<uint4 *>(smem + SM::kD + oh) = dh;
+                    *reinterpret_cast<uint4 *>(smem + SM::kD + ol) = dl;
+                    *reinterpret_cast<uint4 *>(smem + SM::kE + oh) = eh;
+                    *reinterpret_cast<uint4 *>(smem + SM::kE + ol) = el;
                 }
+                if (tid == 64) CHAIN_TS(22);
                 fence_async_shared();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(dd_bar);
+                if (lane == 0) mbar_arrive(d_bar);
                 if (tid == 64) CHAIN_TS(11);
-            } else {
-                // E = dkk Delta from the X warps' Delta
-                wait_on(delta_bar, dl_phase);
-                dl_phase ^= 1;
-                if (tid == 0) CHAIN_TS(20);
-                if (*abort_s) break;
-                float d[16];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 u = *reinterpret_cast<const float4 *>(ureg + uo[q]);
-                    d[4 * q] = dkk * u.x; d[4 * q + 1] = dkk * u.y; d[4 * q + 2] = dkk * u.z; d[4 * q + 3] = dkk * u.w;
-                }
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const float *x = d + 8 * hh;
-                    uint4 eh, el;
-                    split2(x[0], x[1], eh.x, el.x); split2(x[2], x[3], eh.y, el.y);
-                    split2(x[4], x[5], eh.z, el.z); split2(x[6], x[7], eh.w, el.w);
-                    *reinterpret_cast<uint4 *>(smem + SM::kE + dof[hh]) = eh;
-                    *reinterpret_cast<uint4 *>(smem + SM::kE + dof[2 + hh]) = el;
-                }
-                fence_async_shared();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(e_bar);
-                if (tid == 0) CHAIN_TS(22);
             }
-            // ---- S <- ds S + K^T E (two token halves, hi + lo each) -------------------
+            // ---- S <- ds S + K^T E (hi + lo; two token halves when split) --------
             wait_on(s_bar, s_phase);
             s_phase ^= 1;
             if (tid == 64) CHAIN_TS(12);
@@ -465,29 +508,37 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             if (*abort_s) break;
             tc_fence_after();
             {
-                float s0[16], s1[16], s2[16], s3[16];
-                tmem_ld16(tmem + lane_base + kColS + n0, s0);
-                tmem_ld16(tmem + lane_base + kColS + NS + n0, s1);
-                tmem_ld16(tmem + lane_base + kColXB + n0, s2);
-                tmem_ld16(tmem + lane_base + kColXB + NS + n0, s3);
+                float s0[NC], s1[NC], s2[NC], s3[NC];
+                tmem_ld_cols<NC>(tmem + lane_base + kColS + n0, s0);
+                tmem_ld_cols<NC>(tmem + lane_base + kColS + NS + n0, s1);
+                if (kSplitS) {
+                    tmem_ld_cols<NC>(tmem + lane_base + kColSB + n0, s2);
+                    tmem_ld_cols<NC>(tmem + lane_base + kColSB + NS + n0, s3);
+                }
                 tmem_wait_ld();
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int n = 8 * hh;
+                for (int n = 0; n < NC; n += 8) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        S[n + e] = fmaf(ds, S[n + e], (s0[n + e] + s1[n + e]) + (s2[n + e] + s3[n + e]));
+                    for (int e = 0; e < 8; ++e) {
+                        const float dS = kSplitS ? (s0[n + e] + s1[n + e]) + (s2[n + e] + s3[n + e])
+                                                 : s0[n + e] + s1[n + e];
+                        S[n + e] = fmaf(ds, S[n + e], dS);
+                    }
                     uint4 hi, lo;
                     split2(S[n], S[n + 1], hi.x, lo.x); split2(S[n + 2], S[n + 3], hi.y, lo.y);
                     split2(S[n + 4], S[n + 5], hi.z, lo.z); split2(S[n + 6], S[n + 7], hi.w, lo.w);
-                    *reinterpret_cast<uint4 *>(smem + SM::kSL + so[hh]) = hi;
-                    *reinterpret_cast<uint4 *>(smem + SM::kSL + so[2 + hh]) = lo;
+                    *reinterpret_cast<uint4 *>(smem + SM::kSL + sl_off(n0 + n, d_row)) = hi;
+                    *reinterpret_cast<uint4 *>(smem + SM::kSL + sl_off(NS + n0 + n, d_row)) = lo;
                 }
             }
             fence_async_shared();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(r_bar);
+#ifdef GDN_CHAIN_TIMING
+            if (lane == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && step >= 10 && step < 20)
+                g_chain_rarr[step - 10][warp] = clock64();
+#endif
             if (tid == 64) CHAIN_TS(13);
             if (tid == 0) CHAIN_TS(17);
             if (xrows) continue;
@@ -496,82 +547,51 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             pd_phase ^= 1;
             if (*abort_s) break;
             tc_fence_after();
-            float p0[16], p1[16];
-            tmem_ld16(tmem + lane_base + kColPD + n0, p0);
-            tmem_ld16(tmem + lane_base + kColPD + NS + n0, p1);
+            float p0[NC], p1[NC];
+            tmem_ld_cols<NC>(tmem + lane_base + kColPD + n0, p0);
+            tmem_ld_cols<NC>(tmem + lane_base + kColPD + NS + n0, p1);
             tmem_wait_ld();
             if (tid == 0) CHAIN_TS(18);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(pd_free);
-            float4 v[4];
+            float4 v[NC / 4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                v[q].x = fmaf(dq, acc[4 * q], p0[4 * q] + p1[4 * q]);
-                v[q].y = fmaf(dq, acc[4 * q + 1], p0[4 * q + 1] + p1[4 * q + 1]);
-                v[q].z = fmaf(dq, acc[4 * q + 2], p0[4 * q + 2] + p1[4 * q + 2]);
-                v[q].w = fmaf(dq, acc[4 * q + 3], p0[4 * q + 3] + p1[4 * q + 3]);
+            for (int q = 0; q < NC / 4; ++q) {
+                v[q].x = fmaf(dg, acc[4 * q], p0[4 * q] + p1[4 * q]);
+                v[q].y = fmaf(dg, acc[4 * q + 1], p0[4 * q + 1] + p1[4 * q + 1]);
+                v[q].z = fmaf(dg, acc[4 * q + 2], p0[4 * q + 2] + p1[4 * q + 2]);
+                v[q].w = fmaf(dg, acc[4 * q + 3], p0[4 * q + 3] + p1[4 * q + 3]);
             }
-            if (out.mode == kOutStore) {
-                // stage the tile over this stage's U region (its Delta has been read)
-                // as 128B-swizzled boxes of 128-byte rows; issuer C stores it
-                if (sizeof(Tout) == 4) {
+            // stage the tile over this stage's U region (read by now) for issuer C;
+            // the two directions of a bidirectional scan add up in fp32
+            if (sizeof(Tout) == 4 || out.mode == kOutPair) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) *reinterpret_cast<float4 *>(ureg + oo[q]) = v[q];
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 4; q += 2) {
-                        uint4 w;
-                        w.x = pack_bf16(v[q].x, v[q].y); w.y = pack_bf16(v[q].z, v[q].w);
-                        w.z = pack_bf16(v[q + 1].x, v[q + 1].y); w.w = pack_bf16(v[q + 1].z, v[q + 1].w);
-                        *reinterpret_cast<uint4 *>(ureg + oo[q]) = w;
-                    }
-                }
-                fence_async_shared();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(o_bar);
-                    mbar_arrive(&free_st[buf]);
-                }
+                for (int q = 0; q < NC / 4; ++q)
+                    *reinterpret_cast<float4 *>(ureg + out_stage_off<NS, float>(r, n0 + 4 * q)) = v[q];
             } else {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&free_st[buf]);
-                // pair mode: publish this direction's piece; the second finisher combines
-                const int t = c * 64 + r;
-                const size_t off = (((size_t)b * T + (t < T ? t : 0)) * H + h) * DV + j0 + n0;
-                float *mine = dir ? out.part[1] : out.part[0];
-                float *other = dir ? out.part[0] : out.part[1];
-                if (t < T) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) *reinterpret_cast<float4 *>(mine + off + 4 * q) = v[q];
+                for (int q = 0; q < NC / 4; q += 2) {
+                    uint4 w;
+                    w.x = pack_bf16(v[q].x, v[q].y); w.y = pack_bf16(v[q].z, v[q].w);
+                    w.z = pack_bf16(v[q + 1].x, v[q + 1].y); w.w = pack_bf16(v[q + 1].z, v[q + 1].w);
+                    *reinterpret_cast<uint4 *>(ureg + out_stage_off<NS, Tout>(r, n0 + 4 * q)) = w;
                 }
-                __threadfence();
-                __syncwarp();
-                unsigned int prior = 0;
-                if (lane == 0) {
-                    const size_t piece = (((size_t)bh * nC + c) * gridDim.x + slice) * 8 + quarter * 4 + cg;
-                    prior = atomicAdd(out.cnt + piece, 1u);
-                }
-                prior = __shfl_sync(0xffffffffu, prior, 0);
-                if (prior == 1u) {
-                    __threadfence();
-                    if (t < T) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float4 w = __ldcg(reinterpret_cast<const float4 *>(other + off + 4 * q));
-                            float4 sum = v[q];
-                            sum.x += w.x; sum.y += w.y; sum.z += w.z; sum.w += w.w;
-                            store4<Tout>(out.o + off + 4 * q, sum);
-                        }
-                    }
-                }
+            }
+            fence_async_shared();
+            // o_bar completes one phase per tile: not before the storer has seen the last
+            if (step > 0) { wait_on(o_seen, os_phase); os_phase ^= 1; }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(o_bar);
+                mbar_arrive(&free_st[buf]);
             }
             if (tid == 0) CHAIN_TS(19);
         }
         if (!*abort_s && state_out) {
             float *dst = state_out + ((size_t)bh * kDK + d_row) * DV + j0 + n0;
 #pragma unroll
-            for (int n = 0; n < 16; n += 4)
+            for (int n = 0; n < NC; n += 4)
                 *reinterpret_cast<float4 *>(dst + n) = make_float4(S[n], S[n + 1], S[n + 2], S[n + 3]);
         }
     }

@@ -21,17 +21,24 @@ namespace tc2 {
 using namespace gdn::sm100;
 
 constexpr int kDK = 128;                     // key dimension of the tensor-core path
-constexpr uint32_t kWaitTries = 1u << 24;    // bounded mbarrier polls
+constexpr uint32_t kWaitTries = 1u << 24;    // bounded mbarrier polls (try_wait)
+constexpr uint32_t kSpinTries = 1u << 28;    // bounded test_wait spins (~seconds)
 
-// Width of the U slices in the record (columns of d_v): one chain CTA's slice.
-constexpr int kSliceCols = 64;
+// Granule of the U layout in the record (columns of d_v); a chain CTA's
+// slice is a whole number of granules.
+constexpr int kSliceCols = 32;
 
-// Byte offset of U[row][col] inside one 64 x 64 fp32 slice: 256-byte rows
+// Byte offset of U[row][col] inside one 64 x 32 fp32 granule: 128-byte rows
 // whose 16-byte chunks are XOR-swizzled with row % 8, so that eight threads
 // reading the same columns of eight consecutive rows hit distinct banks.
 __host__ __device__ constexpr int u_off(int row, int col) {
-    return row * 256 + ((((col >> 2) ^ (row & 7)) & 15) << 4) + (col & 3) * 4;
+    return row * 128 + ((((col >> 2) ^ row) & 7) << 4) + (col & 3) * 4;
 }
+
+// 128B / 64B swizzle of a byte offset inside a 1024-aligned tile, as TMA
+// applies it (16-byte chunk bits XORed with the 128-byte row bits).
+__device__ __forceinline__ int swz128(int L) { return L ^ (((L >> 7) & 7) << 4); }
+__device__ __forceinline__ int swz64(int L) { return L ^ (((L >> 7) & 3) << 4); }
 
 // Per-chunk record written by the prep kernel and read by the chain kernel,
 // rows in FORWARD token order for either direction (the reverse direction's
@@ -41,7 +48,7 @@ __host__ __device__ constexpr int u_off(int row, int col) {
 //       it stacks under the Q tile into one M=128 operand
 //   Ph  bf16, 64 x 64, 128B-swizzled K-major image                  8192 B
 //   Pl  bf16, same layout (P - Ph)                                 8192 B
-//   U   fp32, [DV/64] slices of 64 x 64, rows swizzled (u_off)    256*DV B
+//   U   fp32, [DV/32] granules of 64 x 32, rows swizzled (u_off)  256*DV B
 //   dq[64], dkk[64], ds, padding                                   1024 B
 // so that a chain CTA fetches its operands with a handful of bulk copies.
 template <int DV>

@@ -353,7 +353,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 const int col = half * (DV / 2) + q * 16;
                 tmem_ld16(tmem + lane_base + kPrepColU + col, u);
                 tmem_wait_ld();
-                if (row_lane) {   // slice col/64, row f, columns col%64 .. +15
+                if (row_lane) {   // granule col/32, row f, columns col%32 .. +15
                     unsigned char *sl = rec + RC::kU + (col / kSliceCols) * RC::kUSlice;
                     const int c0 = col % kSliceCols;
 #pragma unroll
