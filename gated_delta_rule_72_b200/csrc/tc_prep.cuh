@@ -24,6 +24,16 @@
 namespace gdn {
 namespace tc2 {
 
+#ifdef GDN_PREP_TIMING
+// Development aid (not built into the library): cycle stamps of CTA 0's
+// tasks 2..11, thread 0.
+__device__ long long g_prep_ts[10][12];
+#define PREP_TS(slot) do { if (blockIdx.x == 0 && tid == 0 && (t / gridDim.x) >= 2 && (t / gridDim.x) < 12) \
+    g_prep_ts[t / gridDim.x - 2][slot] = clock64(); } while (0)
+#else
+#define PREP_TS(slot) do { } while (0)
+#endif
+
 template <int DV>
 struct PrepSmem {
     static constexpr int kKQ = 32768;                 // [K|Q] x 2 column blocks, 128B swizzle
@@ -36,17 +46,20 @@ struct PrepSmem {
     static constexpr int kT2h = kT1 + 8192;
     static constexpr int kT2l = kT2h + 8192;
     static constexpr int kGate = kT2l + 8192;         // g, beta, dq, dkk, beta e^g
-    static constexpr int kBar = kGate + 5 * 256;      // tma, mma
-    static constexpr int kCtl = kBar + 16;            // tmem base, abort, ds
+    static constexpr int kBar = kGate + 5 * 256;      // tma, mma, gram
+    static constexpr int kCtl = kBar + 32;            // tmem base, abort, ds
     static constexpr int kBytes = kCtl + 16;
     static constexpr int kAlloc = kBytes + 1024;
-    static_assert(kStage % 1024 == 0, "the stage must stay 1024-aligned");
+    static_assert(kStage % 1024 == 0 && kT1 % 1024 == 0, "swizzled areas stay 1024-aligned");
+    // record staging: P and W images over T1 | T2h, U over L | T, gates over T2l
+    static_assert(kT2h == kT1 + 8192 && 64 * DV * 4 <= 2 * 64 * 65 * 4, "record staging areas");
     static_assert(kAlloc <= 232448 / 2 - 1024, "two CTAs per SM");
 };
 
 constexpr int kPrepThreads = 256;
 constexpr int kPrepCtasPerSm = 2;
-constexpr uint32_t kPrepColG = 0;      // 128 lanes x 64 (dead before W is written)
+constexpr uint32_t kPrepColG = 0;      // 128 lanes x 64, first K half (dead before W is written)
+constexpr uint32_t kPrepColG2 = 64;    // second K half
 constexpr uint32_t kPrepColW = 0;      // M=64 x 128
 constexpr uint32_t kPrepColU = 128;    // M=64 x DV
 constexpr uint32_t kPrepTmemCols = 256;
@@ -73,6 +86,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     float *bg_s = g_s + 256;
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + SM::kBar);
     uint64_t *mma_bar = tma_bar + 1;
+    uint64_t *g_bar = tma_bar + 2;     // the two K halves of the Gram product
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + SM::kCtl);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + SM::kCtl + 4);
     float *ds_s = reinterpret_cast<float *>(smem + SM::kCtl + 8);
@@ -87,6 +101,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     if (tid == 0) {
         mbar_init(tma_bar, 1);
         mbar_init(mma_bar, 1);
+        mbar_init(g_bar, 2);
         fence_mbar_init();
         *abort_s = 0;
         prefetch_tensormap(&tm_k);
@@ -142,7 +157,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     if (t < ntasks && tid == 0) issue_tma(t);
     float la_n = 0.f, bt_n = 0.f;
     if (t < ntasks && tid < 64) load_gates(t, la_n, bt_n);
-    uint32_t tma_phase = 0, mma_phase = 0;
+    uint32_t tma_phase = 0, mma_phase = 0, g_phase = 0;
     const uint32_t st_addr = sbase;
 
     for (; t < ntasks; t += gridDim.x) {
@@ -156,6 +171,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         wait_all(tma_bar, tma_phase);
         tma_phase ^= 1;
         __syncthreads();
+        PREP_TS(0);
         if (*abort_s) break;
         if (tn < ntasks && tid < 64) load_gates(tn, la_n, bt_n);   // next task's gates travel meanwhile
         if (warp == 0) {  // inclusive prefix sum of log alpha, 2 rows per lane
@@ -178,27 +194,40 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             bg_s[tid] = beta_s[tid] * __expf(gr);
             if (tid == 0) *ds_s = __expf(gl);
         }
-        // ---- [K; Q] K^T -------------------------------------------------------
-        if (tid == 0) {
+        // ---- [K; Q] K^T, the two K halves from two issuing threads ----------------
+        if (tid == 0 || tid == 32) {
+            const int part = tid >> 5;
             tc_fence_after();
             constexpr uint32_t id = idesc(128, 64, 1, 0, 0);
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint32_t a = st_addr + (s >> 2) * 16384 + (s & 3) * 32;
-                mma_bf16(tmem + kPrepColG, sdesc_sw128(a), sdesc_sw128(a), id, s > 0);
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t a = st_addr + part * 16384 + k * 32;
+                mma_bf16(tmem + (part ? kPrepColG2 : kPrepColG), sdesc_sw128(a), sdesc_sw128(a), id, k > 0);
             }
-            mma_commit(mma_bar);
+            mma_commit(g_bar);
         }
-        wait_all(mma_bar, mma_phase);
-        mma_phase ^= 1;
+        // the previous task's record stores must have read the staging areas
+        if (tid == 0) bulk_wait_read_all();
+        wait_all(g_bar, g_phase);
+        g_phase ^= 1;
+        PREP_TS(2);
         tc_fence_after();
         __syncthreads();  // gate vectors ready
-        // ---- L (fp32, to shared) and P (hi/lo, to the record) ------------------------
+        PREP_TS(1);
+        // ---- L (fp32, to shared) and P (hi/lo images, staged for a bulk store) -------
         {
             float G[32];
-            tmem_ld16(tmem + lane_base + kPrepColG + half * 32, G);
-            tmem_ld16(tmem + lane_base + kPrepColG + half * 32 + 16, G + 16);
-            tmem_wait_ld();
+            {
+                float G2[32];
+                tmem_ld16(tmem + lane_base + kPrepColG + half * 32, G);
+                tmem_ld16(tmem + lane_base + kPrepColG + half * 32 + 16, G + 16);
+                tmem_ld16(tmem + lane_base + kPrepColG2 + half * 32, G2);
+                tmem_ld16(tmem + lane_base + kPrepColG2 + half * 32 + 16, G2 + 16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) G[e] += G2[e];
+            }
+            PREP_TS(9);
             const int ln = quarter * 32 + lane;          // TMEM lane = Gram row
             const int fl = ln & 63;                      // forward row within the chunk
             const int r = rev ? 63 - fl : fl;            // processing row
@@ -228,13 +257,20 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     split2(v[4], v[5], hi.z, lo.z);
                     split2(v[6], v[7], hi.w, lo.w);
                     const int off = sw128(fl, f0 + cc * 8, 0);
-                    *reinterpret_cast<uint4 *>(rec + RC::kPh + off) = hi;
-                    *reinterpret_cast<uint4 *>(rec + RC::kPl + off) = lo;
+                    *reinterpret_cast<uint4 *>(smem + SM::kT1 + off) = hi;          // the record's
+                    *reinterpret_cast<uint4 *>(smem + SM::kT1 + 8192 + off) = lo;   // P_hi | P_lo
                 }
+                fence_async_shared();
             }
         }
+        PREP_TS(10);
         tc_fence_before();
         __syncthreads();
+        if (tid == 0) {
+            bulk_store(rec + RC::kPh, smem + SM::kT1, 16384);
+            bulk_commit_group();
+        }
+        PREP_TS(3);
         // ---- T = (I + L)^{-1}, blocked 16 x 16 (processing order) ------------------
         if (tid < 64) {
             const int blk = tid >> 4, j = tid & 15, o0 = blk * 16;
@@ -255,31 +291,48 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             }
         }
         __syncthreads();
+        PREP_TS(4);
+        // off-diagonal blocks by bands: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj, i = j + band,
+        // each thread a 2 x 2 tile (independent accumulators, conflict-free loads)
         for (int band = 1; band < 4; ++band) {
             const int nblk = 4 - band;
-            for (int e = tid; e < nblk * 256; e += kPrepThreads) {
-                const int j = e >> 8, ii = (e >> 4) & 15, jj = e & 15;
+            for (int e = tid; e < nblk * 64; e += kPrepThreads) {
+                const int j = e >> 6, ti = (e >> 3) & 7, tj = e & 7;
                 const int i = j + band;
-                float acc = 0.f;
-                for (int k = j; k < i; ++k) {
-#pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        acc = fmaf(Lsm[(i * 16 + ii) * 65 + k * 16 + m], Tsm[(k * 16 + m) * 65 + j * 16 + jj], acc);
+                const int a = i * 16 + 2 * ti, bc = j * 16 + 2 * tj;
+                float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+                for (int m = j * 16; m < i * 16; ++m) {
+                    const float l0 = Lsm[a * 65 + m], l1 = Lsm[(a + 1) * 65 + m];
+                    const float t0 = Tsm[m * 65 + bc], t1 = Tsm[m * 65 + bc + 1];
+                    x00 = fmaf(l0, t0, x00); x01 = fmaf(l0, t1, x01);
+                    x10 = fmaf(l1, t0, x10); x11 = fmaf(l1, t1, x11);
                 }
-                Xsm[j * 256 + ii * 16 + jj] = acc;
+                float *xb = Xsm + j * 256 + (2 * ti) * 16 + 2 * tj;
+                xb[0] = x00; xb[1] = x01; xb[16] = x10; xb[17] = x11;
             }
             __syncthreads();
-            for (int e = tid; e < nblk * 256; e += kPrepThreads) {
-                const int j = e >> 8, ii = (e >> 4) & 15, jj = e & 15;
+            for (int e = tid; e < nblk * 64; e += kPrepThreads) {
+                const int j = e >> 6, ti = (e >> 3) & 7, tj = e & 7;
                 const int i = j + band;
-                float acc = 0.f;
+                const int a = i * 16 + 2 * ti, bc = j * 16 + 2 * tj;
+                const float *xb = Xsm + j * 256 + 2 * tj;
+                float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc = fmaf(Tsm[(i * 16 + ii) * 65 + i * 16 + m], Xsm[j * 256 + m * 16 + jj], acc);
-                Tsm[(i * 16 + ii) * 65 + j * 16 + jj] = -acc;
+                for (int m = 0; m < 16; ++m) {
+                    const float t0 = Tsm[a * 65 + i * 16 + m], t1 = Tsm[(a + 1) * 65 + i * 16 + m];
+                    const float x0 = xb[m * 16], x1 = xb[m * 16 + 1];
+                    y00 = fmaf(t0, x0, y00); y01 = fmaf(t0, x1, y01);
+                    y10 = fmaf(t1, x0, y10); y11 = fmaf(t1, x1, y11);
+                }
+                Tsm[a * 65 + bc] = -y00; Tsm[a * 65 + bc + 1] = -y01;
+                Tsm[(a + 1) * 65 + bc] = -y10; Tsm[(a + 1) * 65 + bc + 1] = -y11;
             }
             __syncthreads();
         }
+        // the P store has read its staging area (the T images go there next)
+        if (tid == 0) bulk_wait_read_all();
+        __syncthreads();
+        PREP_TS(5);
         // ---- A operands T diag(beta e^g) (bf16) and T diag(beta) (hi/lo pair), in
         //      forward row/column order (mirrored for the reverse direction) --------
         for (int cell = tid; cell < 64 * 8; cell += kPrepThreads) {
@@ -305,6 +358,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         }
         fence_async_shared();
         __syncthreads();
+        PREP_TS(6);
         // ---- W = T1 K and U = T2 V on the tensor cores (K and V straight from the tiles)
         if (tid == 0) {
             tc_fence_after();
@@ -323,60 +377,74 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             mma_commit(mma_bar);
         }
         wait_all(mma_bar, mma_phase);
+        PREP_TS(7);
         mma_phase ^= 1;
         tc_fence_after();
         // the tiles are consumed: fetch the next task's while this one is written out
         if (tn < ntasks && tid == 0) issue_tma(tn);
-        // ---- record: W (bf16 image), U (fp32 rows), gate vectors ------------------
+        // ---- record: W image, U granules and gate vectors, staged in the areas the
+        //      products are done with (T images, L/T) and written by bulk stores -------
         {
             const bool row_lane = lane < 16;
             const int f = quarter * 16 + lane;       // forward row (M=64 accumulator layout)
+            {
+                float w[64];                         // W columns half*64 .. +63
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {            // W columns half*64 .. +63
-                float w[16];
-                tmem_ld16(tmem + lane_base + kPrepColW + half * 64 + q * 16, w);
+                for (int q = 0; q < 4; ++q) tmem_ld16(tmem + lane_base + kPrepColW + half * 64 + q * 16, w + 16 * q);
                 tmem_wait_ld();
                 if (row_lane) {
-                    uint4 p0, p1;
-                    p0.x = pack_bf16(w[0], w[1]); p0.y = pack_bf16(w[2], w[3]);
-                    p0.z = pack_bf16(w[4], w[5]); p0.w = pack_bf16(w[6], w[7]);
-                    p1.x = pack_bf16(w[8], w[9]); p1.y = pack_bf16(w[10], w[11]);
-                    p1.z = pack_bf16(w[12], w[13]); p1.w = pack_bf16(w[14], w[15]);
-                    const int d0 = half * 64 + q * 16;
-                    *reinterpret_cast<uint4 *>(rec + RC::kW + sw128(f, d0, 8192)) = p0;
-                    *reinterpret_cast<uint4 *>(rec + RC::kW + sw128(f, d0 + 8, 8192)) = p1;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint4 p;
+                        p.x = pack_bf16(w[8 * q], w[8 * q + 1]); p.y = pack_bf16(w[8 * q + 2], w[8 * q + 3]);
+                        p.z = pack_bf16(w[8 * q + 4], w[8 * q + 5]); p.w = pack_bf16(w[8 * q + 6], w[8 * q + 7]);
+                        *reinterpret_cast<uint4 *>(smem + SM::kT1 + sw128(f, half * 64 + 8 * q, 8192)) = p;
+                    }
                 }
             }
 #pragma unroll
-            for (int q = 0; q < DV / 32; ++q) {      // U columns half*DV/2 .. +DV/2-1
-                float u[16];
-                const int col = half * (DV / 2) + q * 16;
+            for (int q2 = 0; q2 < DV / 64; ++q2) {   // U columns half*DV/2 .. +DV/2-1, 32 at a time
+                float u[32];
+                const int col = half * (DV / 2) + q2 * 32;
                 tmem_ld16(tmem + lane_base + kPrepColU + col, u);
+                tmem_ld16(tmem + lane_base + kPrepColU + col + 16, u + 16);
                 tmem_wait_ld();
-                if (row_lane) {   // granule col/32, row f, columns col%32 .. +15
-                    unsigned char *sl = rec + RC::kU + (col / kSliceCols) * RC::kUSlice;
-                    const int c0 = col % kSliceCols;
+                if (row_lane) {   // granule col/32, row f
+                    unsigned char *sl = smem + SM::kL + (col / kSliceCols) * RC::kUSlice;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        *reinterpret_cast<float4 *>(sl + u_off(f, c0 + 4 * i)) =
+                    for (int i = 0; i < 8; ++i)
+                        *reinterpret_cast<float4 *>(sl + u_off(f, 4 * i)) =
                             make_float4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
                 }
             }
             if (tid < 64) {
                 const int r = rev ? 63 - tid : tid;   // record row tid <- processing row r
-                float *gate = reinterpret_cast<float *>(rec + RC::kGate);
+                float *gate = reinterpret_cast<float *>(smem + SM::kT2l);
                 gate[tid] = dq_s[r];
                 gate[64 + tid] = dkk_s[r];
-                if (tid == 0) gate[128] = *ds_s;
+                if (tid == 0) {
+                    gate[128] = *ds_s;
+                    gate[129] = gate[130] = gate[131] = 0.f;
+                }
             }
+            fence_async_shared();
         }
         tc_fence_before();
         __syncthreads();
+        if (tid == 0) {
+            bulk_store(rec + RC::kW, smem + SM::kT1, 16384);
+            bulk_store(rec + RC::kU, smem + SM::kL, 64 * DV * 4);
+            bulk_store(rec + RC::kGate, smem + SM::kT2l, RC::kGateCopy);
+            bulk_commit_group();
+        }
+        PREP_TS(8);
     }
 
+    if (tid == 0) bulk_wait_all();   // the record stores have landed
     if (*abort_s) {
         mbar_wait(tma_bar, tma_phase, 64);
         mbar_wait(mma_bar, mma_phase, 64);
+        mbar_wait(g_bar, g_phase, 64);
     }
     tc_fence_before();
     __syncthreads();
