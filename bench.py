@@ -106,6 +106,17 @@ def kernel_algorithmic_bytes(name, w):
     return reads + writes
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per token-head
+# of a kernel, from one ncu capture of a smaller case of the same launch
+# configuration (profiles/ holds the summaries), scaled by the token-heads a
+# launch processes.  Keyed by (kernel, workload); absent means not captured
+# for this kernel as it stands.
+MEASURED_TRAFFIC_PER_TOKEN_HEAD = {
+    ("tc_chain", "stream480"): 184.07e6 / (12 * 8192),   # chain_kernel<128, 32, float>, T = 8192
+    ("tc_prep", "stream480"): 124.97e6 / (12 * 8192),    # prep_kernel<128>, T = 8192
+}
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -252,11 +263,17 @@ def timed(torch, fn, between, steps, dist=None):
 
 
 def max_over_ranks(torch, dist, x, device):
+    """The slowest rank's time (every rank takes part; gloo on the CPU, NCCL on GPUs)."""
     if dist is None:
         return x
     t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_value(n_gpus, units_per_gpu, ms_max):
+    """Whole-job Mtokens/s: the token-heads all ranks processed over the slowest rank's time."""
+    return n_gpus * units_per_gpu / (ms_max * 1e-3) / 1e6
 
 
 # ---------------------------------------------------------------------------
@@ -390,7 +407,7 @@ def main():
     ms = max_over_ranks(torch, dist, ms, device)
 
     units = w.token_heads                          # per GPU per step
-    value = args.gpus * units / (ms * 1e-3) / 1e6
+    value = whole_job_value(args.gpus, units, ms)
 
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
@@ -413,8 +430,10 @@ def main():
             peak = peaks["bf16_tflops"]
             unit = "TFLOP/s"
         total_ms = sum(t for t, _ in ktimes.values())
+        tph = MEASURED_TRAFFIC_PER_TOKEN_HEAD.get((name, w.name))
+        traffic = tph * units_per_launch if tph is not None else None
         roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": None, "kernel": name,
+                "frac": achieved / peak, "traffic": traffic, "kernel": name,
                 "peak_source": "%s (%s)" % (peak_src, "MEASURED_PEAKS.json" if peak_src == "measured"
                                             else "pool fallback"),
                 "kernel_ms_per_launch": per_launch_ms,

@@ -58,27 +58,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Non-blocking test: has the phase with the given parity completed?
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded spin on test_wait: for a lone issuing thread, which would rather
-// burn its warp's issue slots than be suspended past the phase's completion.
-__device__ __forceinline__ bool mbar_spin(uint64_t *bar, uint32_t parity, uint32_t max_polls) {
-    for (uint32_t i = 0; i < max_polls; ++i)
-        if (mbar_test_wait(bar, parity)) return true;
-    return false;
-}
-
 // Bounded wait for the phase with the given parity to complete.  Returns
 // false if it did not complete within max_polls polls (each try_wait may
 // itself block for a hardware-defined interval), so a kernel never hangs.
@@ -131,6 +110,19 @@ __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
     unsigned int v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Spin until *p >= v (acquire), for at most `limit_ns`; false on timeout.
+__device__ __forceinline__ bool spin_until_geq(const unsigned int *p, unsigned int v,
+                                               unsigned long long limit_ns) {
+    const unsigned long long t0 = global_ns();
+    while (ld_acquire_gpu(p) < v)
+        if (global_ns() - t0 > limit_ns) return false;
+    return true;
 }
 // 1-d bulk copy shared -> global, tracked by this thread's bulk async-group.
 __device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {

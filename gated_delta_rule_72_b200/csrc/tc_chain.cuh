@@ -248,13 +248,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             if (err) atomicAdd(err, 1u);
         }
     };
-    // issuing threads spin instead (a suspended try_wait can oversleep the phase)
-    auto spin_on = [&](uint64_t *bar, uint32_t parity) {
-        if (!mbar_spin(bar, parity, kSpinTries)) {
-            *abort_s = 1;
-            if (err) atomicAdd(err, 1u);
-        }
-    };
     auto stage_addr = [&](int step) { return sbase + (step & 1) * SM::kStage; };
     auto gates = [&](int step) { return reinterpret_cast<const float *>(smem + SM::kG + (step & 1) * SM::kGate); };
     auto adv = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
@@ -396,9 +389,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     tile = ((size_t)bh * nC + c) * gridDim.x + slice;
                     if (atomicAdd(out.cnt + tile, 1u) != 0u) {
                         // second: wait for the first one's "landed" mark (+2)
-                        uint32_t n = 0;
-                        while (ld_acquire_gpu(out.cnt + tile) < 3u && ++n < kSpinTries) {}
-                        if (n >= kSpinTries) {
+                        if (!spin_until_geq(out.cnt + tile, 3u, kFlagWaitNs)) {
                             *abort_s = 1;
                             if (err) atomicAdd(err, 1u);
                             break;

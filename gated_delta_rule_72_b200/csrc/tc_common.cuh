@@ -22,7 +22,7 @@ using namespace gdn::sm100;
 
 constexpr int kDK = 128;                     // key dimension of the tensor-core path
 constexpr uint32_t kWaitTries = 1u << 24;    // bounded mbarrier polls (try_wait)
-constexpr uint32_t kSpinTries = 1u << 28;    // bounded test_wait spins (~seconds)
+constexpr unsigned long long kFlagWaitNs = 2000000000ull;   // bound of a wait on another CTA (2 s)
 
 // Granule of the U layout in the record (columns of d_v); a chain CTA's
 // slice is a whole number of granules.

@@ -131,8 +131,8 @@ GDN_API gdn_status gdn_step(const void *q, const void *k, const void *v,
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - Arguments whose gdn_workspace_size(..., bidir = 0) exceeds
  *     GDN_NOALLOC_SCRATCH_BYTES are rejected with GDN_ERR_WORKSPACE before
- *     any launch (for d = 128 and bf16 inputs that is roughly B*H*ceil(T/64)
- *     > 450 chunk-heads).
+ *     any launch (for d_k = d_v = 128 and bf16 inputs, whose workspace is
+ *     one 66,560-byte record per chunk-head, that is B*H*ceil(T/64) > 1,008).
  *   - All calls share the one array and it keeps the last call's contents;
  *     nothing in it needs to start at zero (every scratch byte a call reads
  *     was written earlier by the same call, in stream order).  Calls that

@@ -16,9 +16,11 @@ def _check_heads(o_gpu, inp, heads, mode="causal", s_gpu=None):
     o_ref, s_ref = oracle_heads(inp, heads=heads, mode=mode)
     tol = TOL[inp["q"].dtype]
     err = rel_err(o_gpu[:, :, heads], o_ref)
+    print("parity max|o - o_oracle| / rms(o_oracle) = %.3e (heads %s)" % (err, heads))
     assert np.isfinite(err) and err <= tol, err
     if s_gpu is not None:
         serr = rel_err(s_gpu[:, heads], s_ref)
+        print("parity max|S - S_oracle| / rms(S_oracle) = %.3e" % serr)
         assert serr <= tol, serr
     return err
 
