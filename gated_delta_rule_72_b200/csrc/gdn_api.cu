@@ -310,7 +310,7 @@ gdn_status launch_chain(const Args &a, const CUtensorMap &mk, const CUtensorMap 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
         return GDN_ERR_CUDA;
     gdn::LaunchScope ls(ndir == 2 ? "tc_chain_bidir" : "tc_chain", a.stream);
-    kern<<<dim3(DV / NS, a.B * a.H, ndir), gdn::tc2::kChainThreads, SM::kAlloc, a.stream>>>(
+    kern<<<dim3(DV / NS, a.B * a.H, ndir), gdn::tc2::chain_threads<NS>(), SM::kAlloc, a.stream>>>(
         mk, mq, mo, recs, state_in, state_out, out, a.T, a.H, nC, 0, err);
     return launch_status();
 }

@@ -33,7 +33,9 @@
 //   all                     S <- ds S + K^T E, thread = one row of S
 // Warps 16 and 17 issue [Q;W] S, one K half each, and K^T E (one token half
 // each when TMEM holds two accumulators for it, else warp 16 alone); warp 19
-// issues P D, warp 20 stores the output tiles and warp 18 loads the stages.  The
+// issues P D, warp 20 stores the output tiles and warp 18 loads the stages.
+// (Four streams for [Q;W] S, where TMEM has room, measured slower: the extra
+// TMEM loads in the critical epilogue cost more than the shorter chains save.)  The
 // roles meet on mbarriers, each of which can only complete its next phase
 // after every waiter has observed the previous one.
 //
@@ -81,7 +83,13 @@ struct ChainSmem {
     static constexpr int kSL = 2 * kStage;                 // [S_hi | S_lo], K = 128
     static constexpr int kD = kSL + 128 * 2 * NS * 2;      // [D_hi | D_lo], K = 64
     static constexpr int kE = kD + 64 * 2 * NS * 2;        // [E_hi | E_lo], K = 64
-    static constexpr int kG = kE + 64 * 2 * NS * 2;        // 2 x gates (dq, dkk, ds)
+    // Output staging: two dedicated buffers where there is room (NS = 32), so
+    // that a stage is free for the next load as soon as its operands are used;
+    // else (NS = 64) the tile is staged over the stage's U area once U is read.
+    static constexpr bool kOwnOut = NS == 32;
+    static constexpr int kOBytes = 64 * NS * 4;
+    static constexpr int kO = kE + 64 * 2 * NS * 2;        // [2] output tiles (kOwnOut)
+    static constexpr int kG = kO + (kOwnOut ? 2 * kOBytes : 0);   // 2 x gates (dq, dkk, ds)
     static constexpr int kGate = 528;
     static constexpr int kBar = kG + 2 * kGate;            // mbarriers
     static constexpr int kCtl = kBar + 128;
@@ -94,8 +102,8 @@ struct ChainSmem {
     static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
-constexpr int kChainWarps = 21;
-constexpr int kChainThreads = kChainWarps * 32;
+template <int NS>
+constexpr int chain_threads() { return 21 * 32; }
 
 enum OutMode { kOutStore = 0, kOutPair = 1 };
 
@@ -146,10 +154,10 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float *v) {
     }
 }
 
-// grid (DV/NS, B*H, directions), block kChainThreads.  blockIdx.z + dir0 is
+// grid (DV/NS, B*H, directions), block chain_threads<NS>().  blockIdx.z + dir0 is
 // the direction (0 causal, 1 reverse).
 template <int DV, int NS, typename Tout>
-__global__ void __launch_bounds__(kChainThreads, 1)
+__global__ void __launch_bounds__(chain_threads<NS>(), 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
              const __grid_constant__ CUtensorMap tm_o, const unsigned char *__restrict__ recs,
              const float *__restrict__ state_in, float *__restrict__ state_out, const ChainOut<Tout> out,
@@ -173,6 +181,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     uint64_t *pd_free = bars + 9;      // P D read, 8 Y warps                       (-> C)
     uint64_t *o_bar = bars + 10;       // output tile staged, 8 Y warps             (-> storer)
     uint64_t *o_seen = bars + 11;      // storer has seen o_bar's phase             (-> Y warps)
+    uint64_t *o_free = bars + 12;      // [2] output buffer read by its store (kOwnOut, -> Y warps)
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + SM::kCtl);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + SM::kCtl + 4);
 
@@ -196,8 +205,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
-        mbar_init(&free_st[0], 20);
-        mbar_init(&free_st[1], 20);
+        // 16 warps and the commits of A, B, C; the storer too when the output
+        // tile is staged inside the stage
+        mbar_init(&free_st[0], SM::kOwnOut ? 19 : 20);
+        mbar_init(&free_st[1], SM::kOwnOut ? 19 : 20);
+        mbar_init(&o_free[0], 1);
+        mbar_init(&o_free[1], 1);
         mbar_init(xy_bar, 2);
         mbar_init(d_bar, 8);
         mbar_init(s_bar, kSplitS ? 2 : 1);
@@ -309,8 +322,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint64_t a = sdesc_sw128(st + SM::kQW + part * 16384 + k * 32);
-                    mma_bf16(tmem + colXY, a, adv(dSL, (part * 4 + k) * 2048), idQW, k > 0);
+                    const int s = part * 4 + k;
+                    const uint64_t a = sdesc_sw128(st + SM::kQW + (s >> 2) * 16384 + (s & 3) * 32);
+                    mma_bf16(tmem + colXY, a, adv(dSL, s * 2048), idQW, k > 0);
                 }
                 if (part == 0) CHAIN_TS(6); else CHAIN_TS(8);
                 mma_commit(xy_bar);
@@ -377,12 +391,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             for (int step = 0; step < nC; ++step) {
                 const int buf = step & 1;
                 const int c = chunk_of(step);
-                // the output warps staged the tile over this stage's U region
+                // the output warps staged the tile (own buffer, or the stage's U area)
                 wait_on(o_bar, o_phase);
                 o_phase ^= 1;
                 mbar_arrive(o_seen);   // o_bar may complete its next phase
                 if (*abort_s) break;
-                const unsigned char *ob = smem + buf * SM::kStage + SM::kU;
+                const unsigned char *ob = SM::kOwnOut ? smem + SM::kO + buf * SM::kOBytes
+                                                      : smem + buf * SM::kStage + SM::kU;
                 bool add = false;      // TMA-reduce-add onto the other direction's tile
                 size_t tile = 0;
                 if (out.mode == kOutPair) {
@@ -408,9 +423,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                     tma_store_4d(&tm_o, ob, j0, h, c * 64, b);
                 }
                 bulk_commit_group();
-                bulk_wait_read_all();            // the stage may be reloaded after this
+                bulk_wait_read_all();            // the staging buffer may be reused after this
                 CHAIN_TS(27);
-                mbar_arrive(&free_st[buf]);
+                mbar_arrive(SM::kOwnOut ? &o_free[buf] : &free_st[buf]);
                 if (out.mode == kOutPair && !add) {
                     bulk_wait_all();             // landed in global memory: mark it (+2)
                     fence_proxy_async_global();
@@ -425,7 +440,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         // ============================ epilogue warps (0..15) ========================
         const bool xrows = quarter >= 2;                 // TMEM lanes 64-127 hold X
         const int r = xrows ? d_row - 64 : d_row;        // token row (forward order) of this lane
-        uint32_t full_phases = 0, xy_phase = 0, s_phase = 0, pd_phase = 0, os_phase = 0;
+        uint32_t full_phases = 0, xy_phase = 0, s_phase = 0, pd_phase = 0, os_phase = 0, of_phases = 0;
         for (int step = 0; step < nC; ++step) {
             const int buf = step & 1;
             const int c = chunk_of(step);
@@ -437,6 +452,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             const float *gt = gates(step);
             const float ds = gt[128];
             const float dg = xrows ? gt[64 + r] : gt[r];   // dkk for X rows, dq for Y rows
+            if (SM::kOwnOut && !xrows) {   // Y rows are done with the stage
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&free_st[buf]);
+            }
             // X rows overwrite D below: the previous P D must have read it
             if (xrows && step > 0) { wait_on(pd_bar, pd_phase); pd_phase ^= 1; }
             wait_on(xy_bar, xy_phase);
@@ -554,19 +573,28 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 v[q].z = fmaf(dg, acc[4 * q + 2], p0[4 * q + 2] + p1[4 * q + 2]);
                 v[q].w = fmaf(dg, acc[4 * q + 3], p0[4 * q + 3] + p1[4 * q + 3]);
             }
-            // stage the tile over this stage's U region (read by now) for issuer C;
-            // the two directions of a bidirectional scan add up in fp32
+            // stage the tile for the storer (own double buffer, or over this stage's
+            // U area, which is read by now); both directions of a bidirectional scan
+            // add up in fp32
+            unsigned char *ob = ureg;
+            if (SM::kOwnOut) {
+                ob = smem + SM::kO + buf * SM::kOBytes;
+                if (step >= 2) {   // the store two tiles back has read this buffer
+                    wait_on(&o_free[buf], (of_phases >> buf) & 1u);
+                    of_phases ^= 1u << buf;
+                }
+            }
             if (sizeof(Tout) == 4 || out.mode == kOutPair) {
 #pragma unroll
                 for (int q = 0; q < NC / 4; ++q)
-                    *reinterpret_cast<float4 *>(ureg + out_stage_off<NS, float>(r, n0 + 4 * q)) = v[q];
+                    *reinterpret_cast<float4 *>(ob + out_stage_off<NS, float>(r, n0 + 4 * q)) = v[q];
             } else {
 #pragma unroll
                 for (int q = 0; q < NC / 4; q += 2) {
                     uint4 w;
                     w.x = pack_bf16(v[q].x, v[q].y); w.y = pack_bf16(v[q].z, v[q].w);
                     w.z = pack_bf16(v[q + 1].x, v[q + 1].y); w.w = pack_bf16(v[q + 1].z, v[q + 1].w);
-                    *reinterpret_cast<uint4 *>(ureg + out_stage_off<NS, Tout>(r, n0 + 4 * q)) = w;
+                    *reinterpret_cast<uint4 *>(ob + out_stage_off<NS, Tout>(r, n0 + 4 * q)) = w;
                 }
             }
             fence_async_shared();
@@ -575,7 +603,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(o_bar);
-                mbar_arrive(&free_st[buf]);
+                if (!SM::kOwnOut) mbar_arrive(&free_st[buf]);
             }
             if (tid == 0) CHAIN_TS(19);
         }
