@@ -193,6 +193,25 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             dkk_s[tid] = __expf(gl - gr);
             bg_s[tid] = beta_s[tid] * __expf(gr);
             if (tid == 0) *ds_s = __expf(gl);
+            // Decay factors of the masks without an exponential per entry: for s in
+            // the 16-token block k, e^{g_r - g_s} = e^{g_r - g_16k} e^{g_16k - g_s}.
+            // On the entries the masks keep (16k <= s <= r) the first factor is at
+            // most 1 and the second at most e^(decay over 16 tokens), so both are
+            // finite whenever that decay stays below 80 (else: one exponential per
+            // entry).  (Scratch: the band buffer, unused until the inverse.)
+            const float gqr = rev ? (tid > 0 ? g_s[tid - 1] : 0.f) : gr;
+            Xsm[tid] = __expf(g_s[tid & ~15] - gr);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                Xsm[64 + tid * 4 + k] = __expf(gr - g_s[16 * k]);
+                Xsm[320 + tid * 4 + k] = __expf(gqr - g_s[16 * k]);
+            }
+            if (tid == 0) {
+                bool fast = true;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) fast = fast && (g_s[16 * k] - g_s[16 * k + 15] < 80.f);
+                reinterpret_cast<int *>(Xsm)[576] = fast ? 1 : 0;
+            }
         }
         // ---- [K; Q] K^T, the two K halves from two issuing threads ----------------
         if (tid == 0 || tid == 32) {
@@ -232,15 +251,22 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             const int fl = ln & 63;                      // forward row within the chunk
             const int r = rev ? 63 - fl : fl;            // processing row
             const int f0 = half * 32;                    // forward columns f0 .. f0+31
+            const bool fast = reinterpret_cast<const int *>(Xsm)[576] != 0;   // task-uniform
+            const float *facs = Xsm;                                       // e^{g_16k - g_s}
+            // the 16-token blocks of this thread's 32 columns: first 16, last 16
+            const int kA = rev ? 3 - (f0 >> 4) : (f0 >> 4), kB = rev ? 2 - (f0 >> 4) : (f0 >> 4) + 1;
             if (ln < 64) {
                 const float br = beta_s[r], gr = g_s[r];
+                const float eA = br * Xsm[64 + r * 4 + kA], eB = br * Xsm[64 + r * 4 + kB];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int s = rev ? 63 - (f0 + e) : f0 + e;
-                    Lsm[r * 65 + s] = s < r ? br * __expf(gr - g_s[s]) * G[e] : 0.f;
+                    const float w = fast ? (e < 16 ? eA : eB) * facs[s] : br * __expf(gr - g_s[s]);
+                    Lsm[r * 65 + s] = s < r ? w * G[e] : 0.f;
                 }
             } else {
                 const float gq = rev ? (r > 0 ? g_s[r - 1] : 0.f) : g_s[r];
+                const float eA = Xsm[320 + r * 4 + kA], eB = Xsm[320 + r * 4 + kB];
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     float v[8];
@@ -249,7 +275,8 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                         const int f = f0 + cc * 8 + e;
                         const int s = rev ? 63 - f : f;
                         const bool keep = rev ? (s < r) : (s <= r);
-                        v[e] = keep ? __expf(gq - g_s[s]) * G[cc * 8 + e] : 0.f;
+                        const float w = fast ? (cc < 2 ? eA : eB) * facs[s] : __expf(gq - g_s[s]);
+                        v[e] = keep ? w * G[cc * 8 + e] : 0.f;
                     }
                     uint4 hi, lo;
                     split2(v[0], v[1], hi.x, lo.x);
