@@ -167,3 +167,27 @@ def test_workspace_is_reusable_and_contents_do_not_matter():
     assert torch.equal(o1, o2)
     o_ref, _ = oracle_heads(inp, mode="bidir")
     assert rel_err(o1, o_ref) <= 2e-2
+
+
+@pytest.mark.parametrize("mode", ["causal", "bidir"])
+def test_strong_forgetting_gates(mode):
+    """A stretch of tokens with alpha = e^-8: a 16-token block of it decays by
+    e^-128, beyond where the masks' decay factors can be split into per-block
+    factors, so those chunks take the one-exponential-per-entry path."""
+    B, H, T, d = 1, 3, 300, 128
+    inp = inputs.generate(B, T, H, d, d, "bf16", seed=4242)
+    a = inp["alpha"].clone()
+    a[:, 100:150] = float(np.exp(-8.0))
+    a[:, 200:203] = float(np.exp(-40.0))
+    inp["alpha"] = a
+    dev = to_dev(inp)
+    if mode == "causal":
+        o, s = gdn.scan_causal(dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"])
+    else:
+        o = gdn.scan_bidir(dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"])
+    torch.cuda.synchronize()
+    assert torch.isfinite(o.float()).all()
+    o_ref, s_ref = oracle_heads(inp, mode=mode)
+    assert rel_err(o, o_ref) <= TOL[torch.bfloat16]
+    if mode == "causal":
+        assert rel_err(s, s_ref) <= TOL[torch.bfloat16]
