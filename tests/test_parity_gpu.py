@@ -191,3 +191,29 @@ def test_strong_forgetting_gates(mode):
     assert rel_err(o, o_ref) <= TOL[torch.bfloat16]
     if mode == "causal":
         assert rel_err(s, s_ref) <= TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("mode,o_dtype", [("causal", torch.float32), ("bidir", torch.float32),
+                                          ("causal", torch.bfloat16), ("bidir", torch.bfloat16)])
+def test_many_heads_take_wide_slices(mode, o_dtype):
+    """Enough heads that the chain uses 64-column state slices (B*H*d_v/32 >
+    the SM count), with a ragged last chunk, a state in, and both output
+    dtypes."""
+    B, H, T, d = 2, 40, 200, 128
+    inp = inputs.generate(B, T, H, d, d, "bf16", seed=777)
+    dev = to_dev(inp)
+    if mode == "causal":
+        s0 = _state(B, H, d, d, seed=5)
+        o, s = gdn.scan_causal(dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], s0.cuda(),
+                               out_dtype=o_dtype)
+        o_ref, s_ref = oracle_heads(inp, state_in=s0)
+    else:
+        o = gdn.scan_bidir(dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], out_dtype=o_dtype)
+        o_ref, _ = oracle_heads(inp, mode="bidir")
+    torch.cuda.synchronize()
+    if o_dtype == torch.float32:
+        assert rel_err(o, o_ref) <= TOL[torch.bfloat16]
+    else:
+        assert rel_err_bf16_out(o, o_ref) <= TOL[torch.bfloat16]
+    if mode == "causal":
+        assert rel_err(s, s_ref) <= TOL[torch.bfloat16]
