@@ -272,7 +272,7 @@ gdn_status launch_prep(const Args &a, const CUtensorMap &mk, const CUtensorMap &
     const int grid = (int)(ntasks < slots ? ntasks : slots);
     gdn::LaunchScope ls("tc_prep", a.stream);
     kern<<<grid, gdn::tc2::kPrepThreads, SM::kAlloc, a.stream>>>(mk, mq, mv, a.alpha, a.beta, recs, a.T,
-                                                                 a.H, nC, nbh, 0, ndir, err);
+                                                                 a.H, nC, nbh, ndir, err);
     return launch_status();
 }
 

@@ -28,8 +28,8 @@ namespace tc2 {
 // Development aid (not built into the library): cycle stamps of CTA 0's
 // tasks 2..11, thread 0.
 __device__ long long g_prep_ts[10][12];
-#define PREP_TS(slot) do { if (blockIdx.x == 0 && tid == 0 && (t / gridDim.x) >= 2 && (t / gridDim.x) < 12) \
-    g_prep_ts[t / gridDim.x - 2][slot] = clock64(); } while (0)
+#define PREP_TS(slot) do { if (first_task == 0 && tid == 0 && (t / task_stride) >= 2 && (t / task_stride) < 12) \
+    g_prep_ts[t / task_stride - 2][slot] = clock64(); } while (0)
 #else
 #define PREP_TS(slot) do { } while (0)
 #endif
@@ -64,18 +64,22 @@ constexpr uint32_t kPrepColW = 0;      // M=64 x 128
 constexpr uint32_t kPrepColU = 128;    // M=64 x DV
 constexpr uint32_t kPrepTmemCols = 256;
 
-// grid: persistent (<= tasks), block 256.  Tasks: dir-major, then chunk, then (b,h).
+// One prep pipeline: 256 threads (ptid 0..255) with their own 1024-aligned
+// shared-memory area `smem` (PrepSmem<DV>), 256 TMEM columns from `tmem` and
+// named barrier `bar_id`; it walks tasks first_task, first_task + stride, ...
+// Tasks are ordered the way the chain consumes them: step k holds chunk k of
+// the causal direction and chunk nC-1-k of the reverse one, then (b, h).
+// With `ready` non-null, each record's flag is set (release) once its bulk
+// stores have landed, for a chain kernel that runs alongside.
 template <int DV>
-__global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
-prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-            const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ alpha,
-            const float *__restrict__ beta, unsigned char *__restrict__ recs, int T, int H,
-            int nC, int nbh, int dir0, int ndir, unsigned int *__restrict__ err)
+__device__ __forceinline__ void prep_pipeline(
+    const CUtensorMap *tm_k, const CUtensorMap *tm_q, const CUtensorMap *tm_v,
+    const float *__restrict__ alpha, const float *__restrict__ beta, unsigned char *__restrict__ recs,
+    unsigned int *__restrict__ ready, int T, int H, int nC, int nbh, int ndir, int first_task,
+    int task_stride, unsigned char *smem, uint32_t tmem, int ptid, int bar_id, unsigned int *__restrict__ err)
 {
     using SM = PrepSmem<DV>;
     using RC = Rec<DV>;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float *Lsm = reinterpret_cast<float *>(smem + SM::kL);
     float *Tsm = reinterpret_cast<float *>(smem + SM::kT);
     float *Xsm = reinterpret_cast<float *>(smem + SM::kX);
@@ -87,16 +91,16 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + SM::kBar);
     uint64_t *mma_bar = tma_bar + 1;
     uint64_t *g_bar = tma_bar + 2;     // the two K halves of the Gram product
-    uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + SM::kCtl);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + SM::kCtl + 4);
     float *ds_s = reinterpret_cast<float *>(smem + SM::kCtl + 8);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = ptid, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;                  // TMEM lane quarter of this warp
     const int half = warp >> 2;                    // column half handled by this warp
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t sbase = smem_u32(smem);
     const int ntasks = ndir * nC * nbh;
+    auto psync = [&]() { asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory"); };
 
     if (tid == 0) {
         mbar_init(tma_bar, 1);
@@ -104,23 +108,17 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         mbar_init(g_bar, 2);
         fence_mbar_init();
         *abort_s = 0;
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_v);
+        prefetch_tensormap(tm_k);
+        prefetch_tensormap(tm_q);
+        prefetch_tensormap(tm_v);
     }
-    if (warp == 0) {
-        tmem_alloc(tmem_base_s, kPrepTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_base_s;
+    psync();
 
     auto task_of = [&](int t, int &dir, int &c, int &bh) {
         bh = t % nbh;
-        c = (t / nbh) % nC;
-        dir = dir0 + t / (nbh * nC);
+        const int k = t / (nbh * ndir);
+        dir = (t / nbh) % ndir;
+        c = dir == 0 ? k : nC - 1 - k;
     };
     auto issue_tma = [&](int t) {
         int dir, c, bh;
@@ -128,13 +126,13 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         const int b = bh / H, h = bh % H, t0 = c * 64;
         unsigned char *st = smem;
         mbar_arrive_expect_tx(tma_bar, SM::kStage);
-        tma_load_4d(st, &tm_k, tma_bar, 0, h, t0, b);
-        tma_load_4d(st + 16384, &tm_k, tma_bar, 64, h, t0, b);
-        tma_load_4d(st + 8192, &tm_q, tma_bar, 0, h, t0, b);
-        tma_load_4d(st + 16384 + 8192, &tm_q, tma_bar, 64, h, t0, b);
+        tma_load_4d(st, tm_k, tma_bar, 0, h, t0, b);
+        tma_load_4d(st + 16384, tm_k, tma_bar, 64, h, t0, b);
+        tma_load_4d(st + 8192, tm_q, tma_bar, 0, h, t0, b);
+        tma_load_4d(st + 16384 + 8192, tm_q, tma_bar, 64, h, t0, b);
 #pragma unroll
         for (int vb = 0; vb < DV / 64; ++vb)
-            tma_load_4d(st + SM::kKQ + vb * 8192, &tm_v, tma_bar, vb * 64, h, t0, b);
+            tma_load_4d(st + SM::kKQ + vb * 8192, tm_v, tma_bar, vb * 64, h, t0, b);
     };
     auto wait_all = [&](uint64_t *bar, uint32_t parity) {
         if (!mbar_wait(bar, parity, kWaitTries)) {
@@ -153,24 +151,25 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         bt = tok < T ? beta[off] : 0.f;
     };
 
-    int t = blockIdx.x;
+    int t = first_task;
     if (t < ntasks && tid == 0) issue_tma(t);
     float la_n = 0.f, bt_n = 0.f;
     if (t < ntasks && tid < 64) load_gates(t, la_n, bt_n);
     uint32_t tma_phase = 0, mma_phase = 0, g_phase = 0;
+    unsigned int *pending_flag = nullptr;   // thread 0: ready flag of the last record stored
     const uint32_t st_addr = sbase;
 
-    for (; t < ntasks; t += gridDim.x) {
+    for (; t < ntasks; t += task_stride) {
         int dir, c, bh;
         task_of(t, dir, c, bh);
         const bool rev = dir != 0;
         unsigned char *rec = recs + ((size_t)(dir * nbh + bh) * nC + c) * RC::kBytes;
-        const int tn = t + gridDim.x;
+        const int tn = t + task_stride;
 
         if (tid < 64) { g_s[tid] = la_n; beta_s[tid] = bt_n; }
         wait_all(tma_bar, tma_phase);
         tma_phase ^= 1;
-        __syncthreads();
+        psync();
         PREP_TS(0);
         if (*abort_s) break;
         if (tn < ntasks && tid < 64) load_gates(tn, la_n, bt_n);   // next task's gates travel meanwhile
@@ -186,7 +185,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             g_s[2 * lane] = ex + a0;
             g_s[2 * lane + 1] = ex + a0 + a1;
         }
-        __syncthreads();
+        psync();
         if (tid < 64) {
             const float gr = g_s[tid], gl = g_s[63];
             dq_s[tid] = rev ? (tid > 0 ? __expf(g_s[tid - 1]) : 1.f) : __expf(gr);
@@ -225,13 +224,24 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             }
             mma_commit(g_bar);
         }
-        // the previous task's record stores must have read the staging areas
-        if (tid == 0) bulk_wait_read_all();
+        // the previous task's record stores must have read the staging areas; when
+        // a chain runs alongside, wait for them to land and flag that record
+        if (tid == 0) {
+            if (ready && pending_flag) {
+                bulk_wait_all();
+                fence_proxy_async_global();
+                __threadfence();
+                st_release_gpu(pending_flag, 1u);
+            } else {
+                bulk_wait_read_all();
+            }
+            pending_flag = ready ? ready + (size_t)(dir * nbh + bh) * nC + c : nullptr;
+        }
         wait_all(g_bar, g_phase);
         g_phase ^= 1;
         PREP_TS(2);
         tc_fence_after();
-        __syncthreads();  // gate vectors ready
+        psync();  // gate vectors ready
         PREP_TS(1);
         // ---- L (fp32, to shared) and P (hi/lo images, staged for a bulk store) -------
         {
@@ -292,7 +302,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         }
         PREP_TS(10);
         tc_fence_before();
-        __syncthreads();
+        psync();
         if (tid == 0) {
             bulk_store(rec + RC::kPh, smem + SM::kT1, 16384);
             bulk_commit_group();
@@ -317,7 +327,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 if ((jj >> 4) > (i >> 4)) Tsm[i * 65 + jj] = 0.f;
             }
         }
-        __syncthreads();
+        psync();
         PREP_TS(4);
         // off-diagonal blocks by bands: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj, i = j + band,
         // each thread a 2 x 2 tile (independent accumulators, conflict-free loads)
@@ -337,7 +347,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 float *xb = Xsm + j * 256 + (2 * ti) * 16 + 2 * tj;
                 xb[0] = x00; xb[1] = x01; xb[16] = x10; xb[17] = x11;
             }
-            __syncthreads();
+            psync();
             for (int e = tid; e < nblk * 64; e += kPrepThreads) {
                 const int j = e >> 6, ti = (e >> 3) & 7, tj = e & 7;
                 const int i = j + band;
@@ -354,11 +364,11 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 Tsm[a * 65 + bc] = -y00; Tsm[a * 65 + bc + 1] = -y01;
                 Tsm[(a + 1) * 65 + bc] = -y10; Tsm[(a + 1) * 65 + bc + 1] = -y11;
             }
-            __syncthreads();
+            psync();
         }
         // the P store has read its staging area (the T images go there next)
         if (tid == 0) bulk_wait_read_all();
-        __syncthreads();
+        psync();
         PREP_TS(5);
         // ---- A operands T diag(beta e^g) (bf16) and T diag(beta) (hi/lo pair), in
         //      forward row/column order (mirrored for the reverse direction) --------
@@ -384,7 +394,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             *reinterpret_cast<uint4 *>(smem + SM::kT2l + off) = l2;
         }
         fence_async_shared();
-        __syncthreads();
+        psync();
         PREP_TS(6);
         // ---- W = T1 K and U = T2 V on the tensor cores (K and V straight from the tiles)
         if (tid == 0) {
@@ -457,7 +467,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             fence_async_shared();
         }
         tc_fence_before();
-        __syncthreads();
+        psync();
         if (tid == 0) {
             bulk_store(rec + RC::kW, smem + SM::kT1, 16384);
             bulk_store(rec + RC::kU, smem + SM::kL, 64 * DV * 4);
@@ -467,15 +477,47 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         PREP_TS(8);
     }
 
-    if (tid == 0) bulk_wait_all();   // the record stores have landed
+    if (tid == 0) {
+        bulk_wait_all();   // the record stores have landed
+        if (pending_flag && !*abort_s) {
+            fence_proxy_async_global();
+            __threadfence();
+            st_release_gpu(pending_flag, 1u);
+        }
+    }
     if (*abort_s) {
         mbar_wait(tma_bar, tma_phase, 64);
         mbar_wait(mma_bar, mma_phase, 64);
         mbar_wait(g_bar, g_phase, 64);
     }
     tc_fence_before();
+    psync();
+}
+
+// Standalone prep: grid persistent (<= tasks), block 256, one pipeline per CTA.
+template <int DV>
+__global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
+prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+            const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ alpha,
+            const float *__restrict__ beta, unsigned char *__restrict__ recs, int T, int H,
+            int nC, int nbh, int ndir, unsigned int *__restrict__ err)
+{
+    using SM = PrepSmem<DV>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + SM::kCtl);
+    if ((threadIdx.x >> 5) == 0) {
+        tmem_alloc(tmem_base_s, kPrepTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kPrepTmemCols);
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_s;
+    prep_pipeline<DV>(&tm_k, &tm_q, &tm_v, alpha, beta, recs, nullptr, T, H, nC, nbh, ndir, blockIdx.x,
+                      gridDim.x, smem, tmem, threadIdx.x, 0, err);
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, kPrepTmemCols);
 }
 
 }  // namespace tc2
