@@ -14,6 +14,7 @@
 #include "launch_stats.cuh"
 #include "simt_kernels.cuh"
 #include "tc_chain.cuh"
+#include "tc_fused.cuh"
 #include "tc_prep.cuh"
 
 // Count of bounded device-side waits that gave up (see gdn_device_timeouts).
@@ -190,6 +191,7 @@ size_t plan_workspace(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dty
     if (use_tc(dt, dk, dv)) {
         const size_t nC = (size_t)(T + kChunk - 1) / kChunk;
         size_t bytes = round_up((bidir ? 2 : 1) * (size_t)B * H * nC * tc_record_bytes(dv), 256);
+        bytes += round_up((bidir ? 2 : 1) * (size_t)B * H * nC * sizeof(unsigned int), 256);   // ready flags
         if (bidir) {
             // the two directions add up in fp32: in o itself, or (bf16 o) in a buffer
             if (o_dt == GDN_BF16) bytes += round_up((size_t)B * T * H * dv * sizeof(float), 256);
@@ -283,6 +285,10 @@ int chain_slice_cols(int B, int H, int dv, int ndir) {
     return (long long)B * H * ndir * (dv / 32) <= sm_count() ? 32 : 64;
 }
 
+// Fewest prep CTAs (two pipelines each) worth a fused launch: below this the
+// prep would lag the chains and two launches do better.
+constexpr int kMinFusedPrepCtas = 32;
+
 // o (bf16) <- sum (fp32), n a multiple of 4 elements.
 __global__ void cast_bf16_kernel(const float4 *__restrict__ sum, uint2 *__restrict__ o, size_t n4) {
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
@@ -311,7 +317,7 @@ gdn_status launch_chain(const Args &a, const CUtensorMap &mk, const CUtensorMap 
         return GDN_ERR_CUDA;
     gdn::LaunchScope ls(ndir == 2 ? "tc_chain_bidir" : "tc_chain", a.stream);
     kern<<<dim3(DV / NS, a.B * a.H, ndir), gdn::tc2::chain_threads<NS>(), SM::kAlloc, a.stream>>>(
-        mk, mq, mo, recs, state_in, state_out, out, a.T, a.H, nC, 0, err);
+        mk, mq, mo, recs, state_in, state_out, out, a.T, a.H, nC, err);
     return launch_status();
 }
 
@@ -325,6 +331,54 @@ gdn_status launch_chain_ns(const Args &a, const CUtensorMap &mk, const CUtensorM
     return launch_chain<DV, 64, Tout>(a, mk, mq, recs, nC, ndir, state_in, state_out, out, target, err);
 }
 
+// Prep and chain in one cooperative launch (tc_fused.cuh): n_chain chain CTAs
+// and n_prep CTAs of two prep pipelines each, all resident at once.  Returns
+// GDN_ERR_UNSUPPORTED (nothing launched) when the launch cannot be cooperative.
+template <int DV, int NS, typename Tout>
+gdn_status launch_fused(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq, const CUtensorMap &mv,
+                        unsigned char *recs, unsigned int *ready, int nC, int ndir, int n_chain, int n_prep,
+                        const float *state_in, float *state_out, const gdn::tc2::ChainOut<Tout> &out,
+                        const void *target, unsigned int *err) {
+    const bool f32t = std::is_same<Tout, float>::value || out.mode == gdn::tc2::kOutPair;
+    CUtensorMap mo;
+    if (!encode_map(&mo, target, a.B, a.T, a.H, DV, f32t ? 32 : NS, (f32t || NS == 64) ? 128 : 64, f32t ? 4 : 2))
+        return GDN_ERR_CUDA;
+    auto kern = gdn::tc2::fused_kernel<DV, NS, Tout>;
+    constexpr int smem = gdn::tc2::fused_smem_alloc<DV, NS>();
+    constexpr int threads = gdn::tc2::chain_threads<NS>();
+    static_assert(smem <= 227 * 1024, "fused launch shared memory");
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess ||
+        per_sm < 1 || n_chain + n_prep > per_sm * sm_count())
+        return GDN_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_chain + n_prep);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    gdn::LaunchScope ls("tc_fused", a.stream);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, mo, a.alpha, a.beta, recs, ready, state_in,
+                                             state_out, out, a.T, a.H, nC, a.B * a.H, ndir, n_chain, err);
+    if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorNotSupported) {
+        (void)cudaGetLastError();
+        return GDN_ERR_UNSUPPORTED;
+    }
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+bool cooperative_supported() {
+    int dev = 0, v = 0;
+    return cudaGetDevice(&dev) == cudaSuccess &&
+           cudaDeviceGetAttribute(&v, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && v != 0;
+}
+
 template <int DV, typename Tout>
 gdn_status run_tc(const Args &a, int bidir) {
     CUtensorMap mk, mq, mv;
@@ -335,31 +389,54 @@ gdn_status run_tc(const Args &a, int bidir) {
     unsigned int *err = timeout_counter();
     if (!err) return GDN_ERR_CUDA;
     const int nC = (a.T + kChunk - 1) / kChunk;
+    const int ndir = bidir ? 2 : 1;
     unsigned char *recs = static_cast<unsigned char *>(a.ws);
-    gdn_status s = launch_prep<DV>(a, mk, mq, mv, recs, nC, bidir ? 2 : 1, err);
-    if (s != GDN_OK) return s;
+    unsigned char *p = recs + round_up((size_t)ndir * a.B * a.H * nC * tc_record_bytes(DV), 256);
+    unsigned int *ready = reinterpret_cast<unsigned int *>(p);
+    p += round_up((size_t)ndir * a.B * a.H * nC * sizeof(unsigned int), 256);
     gdn::tc2::ChainOut<Tout> out{};
-    if (!bidir) {
-        out.mode = gdn::tc2::kOutStore;
-        return launch_chain_ns<DV, Tout>(a, mk, mq, recs, nC, 1, a.state_in, a.state_out, out, a.o, err);
-    }
-    // bidirectional: both directions in one launch, adding up in fp32 (in o
-    // itself for an fp32 o, else in a buffer that is then rounded into o)
     constexpr bool f32_out = std::is_same<Tout, float>::value;
-    unsigned char *p = recs + round_up(2 * (size_t)a.B * a.H * nC * tc_record_bytes(DV), 256);
-    const size_t n = (size_t)a.B * a.T * a.H * DV;
     void *target = a.o;
-    if (!f32_out) {
-        target = p;
-        p += round_up(n * sizeof(float), 256);
+    const size_t n = (size_t)a.B * a.T * a.H * DV;
+    if (bidir) {
+        // both directions in one launch, adding up in fp32 (in o itself for an
+        // fp32 o, else in a buffer that is then rounded into o)
+        if (!f32_out) {
+            target = p;
+            p += round_up(n * sizeof(float), 256);
+        }
+        out.mode = gdn::tc2::kOutPair;
+        out.cnt = reinterpret_cast<unsigned int *>(p);
+        if (cudaMemsetAsync(out.cnt, 0, tc_pair_counters(a.B, a.T, a.H, DV) * sizeof(unsigned int), a.stream) !=
+            cudaSuccess)
+            return GDN_ERR_CUDA;
+    } else {
+        out.mode = gdn::tc2::kOutStore;
     }
-    out.mode = gdn::tc2::kOutPair;
-    out.cnt = reinterpret_cast<unsigned int *>(p);
-    if (cudaMemsetAsync(out.cnt, 0, tc_pair_counters(a.B, a.T, a.H, DV) * sizeof(unsigned int), a.stream) !=
-        cudaSuccess)
-        return GDN_ERR_CUDA;
-    s = launch_chain_ns<DV, Tout>(a, mk, mq, recs, nC, 2, nullptr, nullptr, out, target, err);
-    if (s != GDN_OK || f32_out) return s;
+    const float *s_in = bidir ? nullptr : a.state_in;
+    float *s_out = bidir ? nullptr : a.state_out;
+
+    // One cooperative launch (prep on the SMs the chain leaves free) when the
+    // chain grid leaves room for it; else prep, then chain.
+    const int sms = sm_count();
+    const int ns = chain_slice_cols(a.B, a.H, DV, ndir);
+    const long long n_chain = (long long)(DV / ns) * a.B * a.H * ndir;
+    gdn_status s = GDN_ERR_UNSUPPORTED;
+    if (n_chain + kMinFusedPrepCtas <= sms && cooperative_supported()) {
+        if (cudaMemsetAsync(ready, 0, (size_t)ndir * a.B * a.H * nC * sizeof(unsigned int), a.stream) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        const int n_prep = sms - (int)n_chain;
+        s = ns == 32 ? launch_fused<DV, 32, Tout>(a, mk, mq, mv, recs, ready, nC, ndir, (int)n_chain, n_prep, s_in,
+                                                  s_out, out, target, err)
+                     : launch_fused<DV, 64, Tout>(a, mk, mq, mv, recs, ready, nC, ndir, (int)n_chain, n_prep, s_in,
+                                                  s_out, out, target, err);
+    }
+    if (s == GDN_ERR_UNSUPPORTED) {
+        s = launch_prep<DV>(a, mk, mq, mv, recs, nC, ndir, err);
+        if (s != GDN_OK) return s;
+        s = launch_chain_ns<DV, Tout>(a, mk, mq, recs, nC, ndir, s_in, s_out, out, target, err);
+    }
+    if (s != GDN_OK || !bidir || f32_out) return s;
     gdn::LaunchScope ls("tc_bidir_cast", a.stream);
     const size_t n4 = n / 4;
     const int grid = (int)((n4 + 255) / 256 < (size_t)sm_count() * 8 ? (n4 + 255) / 256 : (size_t)sm_count() * 8);

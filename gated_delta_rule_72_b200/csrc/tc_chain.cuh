@@ -58,7 +58,7 @@ namespace tc2 {
 // steps 10..19.
 __device__ long long g_chain_ts[10][32];
 __device__ long long g_chain_rarr[10][20];   // per-warp arrival on the S-rewritten barrier
-#define CHAIN_TS(slot) do { if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && \
+#define CHAIN_TS(slot) do { if (slice == 0 && bh == 0 && dir == 0 && \
     step >= 10 && step < 20) g_chain_ts[step - 10][slot] = clock64(); } while (0)
 #else
 #define CHAIN_TS(slot) do { } while (0)
@@ -103,7 +103,7 @@ struct ChainSmem {
 };
 
 template <int NS>
-constexpr int chain_threads() { return 21 * 32; }
+__host__ __device__ constexpr int chain_threads() { return 21 * 32; }
 
 enum OutMode { kOutStore = 0, kOutPair = 1 };
 
@@ -154,22 +154,23 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float *v) {
     }
 }
 
-// grid (DV/NS, B*H, directions), block chain_threads<NS>().  blockIdx.z + dir0 is
-// the direction (0 causal, 1 reverse).
+// The chain of one (slice, bh, dir): block chain_threads<NS>(), `smem` its
+// 1024-aligned shared memory (ChainSmem<NS>); nslices = DV / NS, nbh = B * H.
+// With `ready` non-null the prep records are produced alongside (by other CTAs
+// of a cooperative launch) and each record's flag is waited for (bounded)
+// before the record is loaded.
 template <int DV, int NS, typename Tout>
-__global__ void __launch_bounds__(chain_threads<NS>(), 1)
-chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-             const __grid_constant__ CUtensorMap tm_o, const unsigned char *__restrict__ recs,
-             const float *__restrict__ state_in, float *__restrict__ state_out, const ChainOut<Tout> out,
-             int T, int H, int nC, int dir0, unsigned int *__restrict__ err)
+__device__ __forceinline__ void chain_body(
+    const CUtensorMap *tm_k, const CUtensorMap *tm_q, const CUtensorMap *tm_o,
+    const unsigned char *__restrict__ recs, const float *__restrict__ state_in, float *__restrict__ state_out,
+    const ChainOut<Tout> &out, const unsigned int *__restrict__ ready, int T, int H, int nC, int slice,
+    int bh, int dir, int nslices, int nbh, unsigned char *smem, unsigned int *__restrict__ err)
 {
     using SM = ChainSmem<NS>;
     using RC = Rec<DV>;
     constexpr int N2 = 2 * NS;          // accumulator width: hi | lo
     constexpr int NC = NS / 4;          // columns per epilogue warp
     constexpr bool kSplitS = 5 * N2 <= 512;   // K^T E in two streams (own TMEM columns)
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kBar);
     uint64_t *full = bars + 0;         // [2] stage loaded                          (loader -> all)
     uint64_t *free_st = bars + 2;      // [2] stage consumed: 16 warps, A, B, C, storer (-> loader)
@@ -187,10 +188,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, cg = (warp >> 2) & 3;
-    const int slice = blockIdx.x, bh = blockIdx.y, dir = dir0 + blockIdx.z;
     const int b = bh / H, h = bh % H;
     const int j0 = slice * NS;
-    const int nbh = gridDim.y;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int n0 = cg * NC;                                 // this warp's columns of the slice
@@ -221,9 +220,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         mbar_init(o_seen, 1);
         fence_mbar_init();
         *abort_s = 0;
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_o);
+        prefetch_tensormap(tm_k);
+        prefetch_tensormap(tm_q);
+        prefetch_tensormap(tm_o);
     }
     if (warp == 0) {
         tmem_alloc(tmem_base_s, kCols);
@@ -283,17 +282,25 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 }
                 if (*abort_s) break;
                 const int c = chunk_of(step);
+                if (ready) {   // the record is prepared alongside: wait until it has landed
+                    if (!spin_until_geq(ready + (size_t)(dir * nbh + bh) * nC + c, 1u, kFlagWaitNs)) {
+                        *abort_s = 1;
+                        if (err) atomicAdd(err, 1u);
+                        break;
+                    }
+                    fence_proxy_async_global();
+                }
                 unsigned char *st = smem + buf * SM::kStage;
                 const unsigned char *rec = rec_base + (size_t)c * RC::kBytes;
                 uint64_t *bar = &full[buf];
                 mbar_arrive_expect_tx(bar, 4 * 16384 + 64 * NS * 4 + SM::kGate);
                 const int t0 = c * 64;
-                tma_load_4d(st + SM::kQW, &tm_q, bar, 0, h, t0, b);
-                tma_load_4d(st + SM::kQW + 16384, &tm_q, bar, 64, h, t0, b);
+                tma_load_4d(st + SM::kQW, tm_q, bar, 0, h, t0, b);
+                tma_load_4d(st + SM::kQW + 16384, tm_q, bar, 64, h, t0, b);
                 bulk_load(st + SM::kQW + 8192, rec + RC::kW, 8192, bar);
                 bulk_load(st + SM::kQW + 16384 + 8192, rec + RC::kW + 8192, 8192, bar);
-                tma_load_4d(st + SM::kK, &tm_k, bar, 0, h, t0, b);
-                tma_load_4d(st + SM::kK + 8192, &tm_k, bar, 64, h, t0, b);
+                tma_load_4d(st + SM::kK, tm_k, bar, 0, h, t0, b);
+                tma_load_4d(st + SM::kK + 8192, tm_k, bar, 64, h, t0, b);
                 bulk_load(st + SM::kP, rec + RC::kPh, 16384, bar);
                 bulk_load(st + SM::kU, rec + RC::kU + j0 * 64 * 4, 64 * NS * 4, bar);
                 bulk_load(smem + SM::kG + buf * SM::kGate, rec + RC::kGate, SM::kGate, bar);
@@ -401,7 +408,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 bool add = false;      // TMA-reduce-add onto the other direction's tile
                 size_t tile = 0;
                 if (out.mode == kOutPair) {
-                    tile = ((size_t)bh * nC + c) * gridDim.x + slice;
+                    tile = ((size_t)bh * nC + c) * nslices + slice;
                     if (atomicAdd(out.cnt + tile, 1u) != 0u) {
                         // second: wait for the first one's "landed" mark (+2)
                         if (!spin_until_geq(out.cnt + tile, 3u, kFlagWaitNs)) {
@@ -416,11 +423,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
                 if (sizeof(Tout) == 4 || out.mode == kOutPair) {
 #pragma unroll
                     for (int x = 0; x < NS / 32; ++x) {
-                        if (add) tma_reduce_add_4d(&tm_o, ob + x * 8192, j0 + 32 * x, h, c * 64, b);
-                        else tma_store_4d(&tm_o, ob + x * 8192, j0 + 32 * x, h, c * 64, b);
+                        if (add) tma_reduce_add_4d(tm_o, ob + x * 8192, j0 + 32 * x, h, c * 64, b);
+                        else tma_store_4d(tm_o, ob + x * 8192, j0 + 32 * x, h, c * 64, b);
                     }
                 } else {
-                    tma_store_4d(&tm_o, ob, j0, h, c * 64, b);
+                    tma_store_4d(tm_o, ob, j0, h, c * 64, b);
                 }
                 bulk_commit_group();
                 bulk_wait_read_all();            // the staging buffer may be reused after this
@@ -546,7 +553,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) mbar_arrive(r_bar);
 #ifdef GDN_CHAIN_TIMING
-            if (lane == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && step >= 10 && step < 20)
+            if (lane == 0 && slice == 0 && bh == 0 && dir == 0 && step >= 10 && step < 20)
                 g_chain_rarr[step - 10][warp] = clock64();
 #endif
             if (tid == 64) CHAIN_TS(13);
@@ -628,6 +635,21 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kCols);
+}
+
+// grid (DV/NS, B*H, directions), block chain_threads<NS>(); blockIdx.z is the
+// direction (0 causal, 1 reverse).
+template <int DV, int NS, typename Tout>
+__global__ void __launch_bounds__(chain_threads<NS>(), 1)
+chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+             const __grid_constant__ CUtensorMap tm_o, const unsigned char *__restrict__ recs,
+             const float *__restrict__ state_in, float *__restrict__ state_out, const ChainOut<Tout> out,
+             int T, int H, int nC, unsigned int *__restrict__ err)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    chain_body<DV, NS, Tout>(&tm_k, &tm_q, &tm_o, recs, state_in, state_out, out, nullptr, T, H, nC, blockIdx.x,
+                             blockIdx.y, blockIdx.z, gridDim.x, gridDim.y, smem, err);
 }
 
 }  // namespace tc2

@@ -1,0 +1,81 @@
+// tc_fused.cuh -- prep and chain in one cooperative launch.
+//
+// When the chain needs fewer CTAs than the GPU has SMs (few heads, long
+// sequences: the chain is latency-bound and most SMs would idle), one launch
+// runs both: CTAs [0, n_chain) are chain CTAs (one state slice each, as in
+// chain_kernel) and every other CTA runs two prep pipelines (each as in
+// prep_kernel, on half of the CTA's shared memory and TMEM).  The prep
+// pipelines walk the chunk tasks in the order the chains consume them and set
+// a ready flag per record once its stores have landed; a chain's loader waits
+// for the flag of each record before fetching it.  The launch is cooperative,
+// so every CTA is resident at once: the prep pipelines never wait on a chain,
+// and a chain only waits on prep pipelines that are running.  Every wait is
+// bounded (a flag wait gives up after kFlagWaitNs and flags an error).
+#pragma once
+
+#include "tc_chain.cuh"
+#include "tc_prep.cuh"
+
+namespace gdn {
+namespace tc2 {
+
+// Shared memory of a prep CTA of the fused launch: two pipeline areas.
+template <int DV>
+struct FusedPrepSmem {
+    static constexpr int kArea = (PrepSmem<DV>::kBytes + 1023) / 1024 * 1024;
+    static constexpr int kCtl = 2 * kArea;          // TMEM base of the CTA
+    static constexpr int kBytes = kCtl + 16;
+};
+
+template <int DV, int NS>
+constexpr int fused_smem_alloc() {
+    return (ChainSmem<NS>::kAlloc > FusedPrepSmem<DV>::kBytes + 1024) ? ChainSmem<NS>::kAlloc
+                                                                       : FusedPrepSmem<DV>::kBytes + 1024;
+}
+
+// grid n_chain + n_prep CTAs (cooperative), block chain_threads<NS>().
+// Chain CTA i: slice i % (DV/NS), (b,h) (i / (DV/NS)) % nbh, direction i / (DV/NS * nbh).
+template <int DV, int NS, typename Tout>
+__global__ void __launch_bounds__(chain_threads<NS>(), 1)
+fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+             const float *__restrict__ alpha, const float *__restrict__ beta, unsigned char *__restrict__ recs,
+             unsigned int *__restrict__ ready, const float *__restrict__ state_in, float *__restrict__ state_out,
+             const ChainOut<Tout> out, int T, int H, int nC, int nbh, int ndir, int n_chain,
+             unsigned int *__restrict__ err)
+{
+    static_assert(chain_threads<NS>() >= 2 * kPrepThreads, "two prep pipelines per CTA");
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int nsl = DV / NS;
+    if ((int)blockIdx.x < n_chain) {
+        const int i = blockIdx.x;
+        chain_body<DV, NS, Tout>(&tm_k, &tm_q, &tm_o, recs, state_in, state_out, out, ready, T, H, nC, i % nsl,
+                                 (i / nsl) % nbh, i / (nsl * nbh), nsl, nbh, smem, err);
+        return;
+    }
+    // ---- two prep pipelines: warps 0-7 and 8-15 (the rest of the block idles)
+    using FS = FusedPrepSmem<DV>;
+    const int warp = threadIdx.x >> 5;
+    uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + FS::kCtl);
+    if (warp == 0) {
+        tmem_alloc(tmem_base_s, 2 * kPrepTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_s;
+    if (warp < 16) {
+        const int pipe = warp >> 3;
+        const int npipes = 2 * ((int)gridDim.x - n_chain);
+        prep_pipeline<DV>(&tm_k, &tm_q, &tm_v, alpha, beta, recs, ready, T, H, nC, nbh, ndir,
+                          2 * ((int)blockIdx.x - n_chain) + pipe, npipes, smem + pipe * FS::kArea,
+                          tmem + pipe * kPrepTmemCols, threadIdx.x & (kPrepThreads - 1), 1 + pipe, err);
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 2 * kPrepTmemCols);
+}
+
+}  // namespace tc2
+}  // namespace gdn
