@@ -122,6 +122,7 @@ __device__ __forceinline__ unsigned long long global_ns() {
 // Spin until *p >= v (acquire), for at most `limit_ns`; false on timeout.
 __device__ __forceinline__ bool spin_until_geq(const unsigned int *p, unsigned int v,
                                                unsigned long long limit_ns) {
+    if (ld_acquire_gpu(p) >= v) return true;
     const unsigned long long t0 = global_ns();
     while (ld_acquire_gpu(p) < v)
         if (global_ns() - t0 > limit_ns) return false;

@@ -276,20 +276,20 @@ __device__ __forceinline__ void chain_body(
             uint32_t free_phases = 0;
             for (int step = 0; step < nC; ++step) {
                 const int buf = step & 1;
+                const int c = chunk_of(step);
+                // the record is prepared alongside: wait until it has landed (polled
+                // before the stage wait, which it then overlaps)
+                if (ready && !spin_until_geq(ready + (size_t)(dir * nbh + bh) * nC + c, 1u, kFlagWaitNs)) {
+                    *abort_s = 1;
+                    if (err) atomicAdd(err, 1u);
+                    break;
+                }
                 if (step >= 2) {   // the stage's previous chunk has been consumed
                     wait_on(&free_st[buf], (free_phases >> buf) & 1u);
                     free_phases ^= 1u << buf;
                 }
                 if (*abort_s) break;
-                const int c = chunk_of(step);
-                if (ready) {   // the record is prepared alongside: wait until it has landed
-                    if (!spin_until_geq(ready + (size_t)(dir * nbh + bh) * nC + c, 1u, kFlagWaitNs)) {
-                        *abort_s = 1;
-                        if (err) atomicAdd(err, 1u);
-                        break;
-                    }
-                    fence_proxy_async_global();
-                }
+                if (ready) fence_proxy_async_global();
                 unsigned char *st = smem + buf * SM::kStage;
                 const unsigned char *rec = rec_base + (size_t)c * RC::kBytes;
                 uint64_t *bar = &full[buf];
