@@ -23,8 +23,9 @@ the measured peak), `cpu_baseline` (the FP64 oracle on a bounded sample, on
 the host cores; rank 0 at N = 1), `e2e` (the same metric through the Python
 API with the inputs copied from pinned host memory and the output and state
 read back inside the timed region), `clocks` (nvidia-smi samples taken during
-the timed region) and `gpu_launches` (kernels the library launched in the
-timed region, from its own launch counter).
+the timed region), `gpu_launches` (kernels the library launched in the
+timed region, from its own launch counter) and, for the rollout workload,
+`graph` (the same step captured once in a CUDA graph and replayed).
 
 `--impl reference` times the FP64 oracle (the reference implementation of
 this build) on the host cores instead: each step is a bounded sample of the
@@ -263,6 +264,21 @@ def timed(torch, fn, between, steps, dist=None):
     return sum(s.elapsed_time(e) for s, e in ev) / steps
 
 
+def graph_replay_ms(torch, step, steps, dist=None):
+    """The rollout's calls captured once in a CUDA graph, then `steps` replays
+    timed like the eager steps (mean device ms per replay)."""
+    g = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        step.run()
+    for _ in range(3):
+        step.between()
+        g.replay()
+    ms = timed(torch, g.replay, step.between, steps, dist)
+    del g
+    return ms
+
+
 def max_over_ranks(torch, dist, x, device):
     """The slowest rank's time (every rank takes part; gloo on the CPU, NCCL on GPUs)."""
     if dist is None:
@@ -448,6 +464,13 @@ def main():
                  "bound": "hbm" if t_mem >= t_flop else "tensor",
                  "frac": max(t_mem, t_flop) / (ms * 1e-3)}
 
+    # ---- the streaming rollout replayed from a CUDA graph (device-timed like value)
+    graph = None
+    if w.mode == "rollout":
+        gms = max_over_ranks(torch, dist, graph_replay_ms(torch, step, args.steps, dist), device)
+        graph = {"value": whole_job_value(args.gpus, units, gms), "unit": UNIT, "ms_per_step": gms,
+                 "calls_per_step": w.calls}
+
     # ---- end to end through the public API, host buffers
     e2e = None
     if not args.no_e2e:
@@ -468,6 +491,8 @@ def main():
                                            else "L2 flushed between steps (256 MB write)")),
                 "roofline": roof, "step_roofline": step_roof,
                 "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches}
+        if graph is not None:
+            line["graph"] = graph
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

@@ -31,6 +31,7 @@ SIGNATURES = {
     "gdn_launch_count": (ctypes.c_ulonglong, []),
     "gdn_device_timeouts": (_I, [ctypes.POINTER(ctypes.c_uint)]),
     "gdn_set_kernel_timing": (None, [_I]),
+    "gdn_set_short_call_tokens": (_I, [_I]),
     "gdn_read_kernel_timing": (_I, [ctypes.c_char_p, _I, ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(_I), _I]),
 }
@@ -114,6 +115,13 @@ def gdn_launch_count():
 
 def gdn_set_kernel_timing(on):
     load().gdn_set_kernel_timing(int(bool(on)))
+
+
+def gdn_set_short_call_tokens(max_t):
+    """Causal calls of at most max_t tokens (at most 64) run token by token;
+    max_t < 0 restores the automatic choice.  Returns the previous setting
+    (-1 for automatic)."""
+    return int(load().gdn_set_short_call_tokens(int(max_t)))
 
 
 def gdn_read_kernel_timing(max_kernels=16, name_len=64):

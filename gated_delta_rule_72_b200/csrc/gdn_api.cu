@@ -6,6 +6,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <type_traits>
 
@@ -16,6 +17,7 @@
 #include "tc_chain.cuh"
 #include "tc_fused.cuh"
 #include "tc_prep.cuh"
+#include "token_step.cuh"
 
 // Count of bounded device-side waits that gave up (see gdn_device_timeouts).
 static __device__ unsigned int g_wait_timeouts;
@@ -450,11 +452,58 @@ gdn_status dispatch_tc(const Args &a, int bidir) {
     return a.o_dt == GDN_F32 ? run_tc<64, float>(a, bidir) : run_tc<64, __nv_bfloat16>(a, bidir);
 }
 
+// ---------------------------------------------------------------------------
+// Short causal calls: token by token (token_step.cuh)
+// ---------------------------------------------------------------------------
+// < 0: automatic (below); else calls of at most this many tokens
+std::atomic<int> g_short_call_tokens{-1};
+
+// Automatic choice, from B200 timings of single calls (d = 128): the token
+// path costs about 2.5 us plus 0.37 us per token for each wave of CTAs
+// (B*H*dv/32 CTAs over the SMs), a one-chunk call of the chunked path about
+// 24 us; so the token path is taken while tokens x waves <= 48.
+bool take_token_path(const Args &a) {
+    const int lim = g_short_call_tokens.load(std::memory_order_relaxed);
+    if (lim >= 0) return a.T <= lim;
+    if (a.T > gdn::tok::kMaxT) return false;
+    const long long ctas = (long long)a.B * a.H * (a.dv / gdn::tok::kCols);
+    const long long waves = (ctas + sm_count() - 1) / sm_count();
+    return (long long)a.T * waves <= 48;
+}
+
+template <int DK, int DV, typename Tin, typename Tout>
+gdn_status run_token(const Args &a) {
+    auto kern = gdn::tok::token_kernel<DK, DV, Tin, Tout>;
+    constexpr int smem = gdn::tok::TokSmem<DK>::kBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    gdn::LaunchScope ls("token_step", a.stream);
+    kern<<<dim3(DV / gdn::tok::kCols, a.B * a.H), gdn::tok::kThreads, smem, a.stream>>>(
+        static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k), static_cast<const Tin *>(a.v), a.alpha,
+        a.beta, a.state_in, a.state_out, static_cast<Tout *>(a.o), a.T, a.H);
+    return launch_status();
+}
+
+template <typename Tin, typename Tout>
+gdn_status token_dims(const Args &a) {
+    if (a.dk == 128 && a.dv == 128) return run_token<128, 128, Tin, Tout>(a);
+    if (a.dk == 128 && a.dv == 64) return run_token<128, 64, Tin, Tout>(a);
+    if (a.dk == 64 && a.dv == 128) return run_token<64, 128, Tin, Tout>(a);
+    return run_token<64, 64, Tin, Tout>(a);
+}
+
+gdn_status run_short(const Args &a) {
+    if (a.dt == GDN_F32)
+        return a.o_dt == GDN_F32 ? token_dims<float, float>(a) : token_dims<float, __nv_bfloat16>(a);
+    return a.o_dt == GDN_F32 ? token_dims<__nv_bfloat16, float>(a) : token_dims<__nv_bfloat16, __nv_bfloat16>(a);
+}
+
 gdn_status run(const Args &a, int bidir) {
     const gdn_status s =
         check_ws(a, plan_workspace(a.B, a.T, a.H, a.dk, a.dv, a.dt, a.o_dt, bidir));
     if (s != GDN_OK) return s;
     if (a.T == 0) return bidir ? GDN_OK : empty_scan(a);
+    if (!bidir && take_token_path(a)) return run_short(a);
     if (use_tc(a.dt, a.dk, a.dv)) return dispatch_tc(a, bidir);
     return a.dt == GDN_F32 ? dispatch_out<float>(a, bidir) : dispatch_out<__nv_bfloat16>(a, bidir);
 }
@@ -580,6 +629,11 @@ int gdn_device_timeouts(unsigned int *count) {
 
 unsigned long long gdn_launch_count(void) {
     return gdn::LaunchStats::get().launches.load(std::memory_order_relaxed);
+}
+
+int gdn_set_short_call_tokens(int max_t) {
+    const int v = max_t < 0 ? -1 : (max_t > gdn::tok::kMaxT ? gdn::tok::kMaxT : max_t);
+    return g_short_call_tokens.exchange(v);
 }
 
 void gdn_set_kernel_timing(int on) { gdn::LaunchStats::get().timing.store(on != 0); }

@@ -154,6 +154,24 @@ GDN_API gdn_status gdn_step_noalloc(const void *q, const void *k, const void *v,
 GDN_API size_t gdn_workspace_size(int B, int T, int H, int dk, int dv, gdn_dtype dt,
                                   gdn_dtype o_dt, int bidir);
 
+/*
+ * gdn_set_short_call_tokens -- which causal calls (gdn_scan_causal, gdn_step,
+ * gdn_step_noalloc) walk their tokens one by one on the CUDA cores, state
+ * slice in registers, in fp32 (the recurrence written out per token:
+ * p = S^T k, S <- alpha S + k (beta (v - alpha p))^T, o = S^T q), instead of
+ * the chunked path.  A short call's fixed cost is then a few microseconds
+ * instead of a chunk prep plus a chain step.  max_t < 0: automatic (the
+ * default): calls of T <= 64 tokens whose T times the number of waves of
+ * their B*H*dv/32 CTAs over the SMs is at most 48 (the measured break-even);
+ * 0: never; 1..64 (larger values clamp to 64): every call of T <= max_t.
+ * Bidirectional calls always take the chunked path.  Returns the previous
+ * setting (-1 for automatic).  The setting is process-wide and read at each
+ * call; it changes which kernels run, not the workspace a call needs
+ * (gdn_workspace_size does not depend on it).  Both paths meet the same
+ * tolerances.
+ */
+GDN_API int gdn_set_short_call_tokens(int max_t);
+
 /* gdn_status_string -- static, NUL-terminated description of a status. */
 GDN_API const char *gdn_status_string(gdn_status s);
 

@@ -141,3 +141,16 @@ def test_noalloc_rejects_oversized_before_launch(lib):
     assert st == -1
     st = _lib.gdn_step_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, 2, 96, 64, 0, 0, None)
     assert st == -5
+
+
+def test_short_call_threshold_is_clamped(lib):
+    """gdn_set_short_call_tokens: negative = automatic (-1, the default), else
+    clamped to at most 64; returns the previous setting (host-side only)."""
+    prev = lib.gdn_set_short_call_tokens(1000)
+    try:
+        assert lib.gdn_set_short_call_tokens(-5) == 64
+        assert lib.gdn_set_short_call_tokens(0) == -1
+        assert lib.gdn_set_short_call_tokens(17) == 0
+        assert lib.gdn_set_short_call_tokens(17) == 17
+    finally:
+        lib.gdn_set_short_call_tokens(prev)

@@ -51,6 +51,57 @@ def test_causal_shapes(dtype, dk, dv, T):
     assert rel_err(s, s_ref) <= tol
 
 
+@pytest.mark.parametrize("path", ["token", "chunked"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", SHAPES)
+@pytest.mark.parametrize("T", [1, 2, 17, 63, 64])
+def test_short_calls_both_paths(path, dtype, dk, dv, T):
+    """Calls of at most 64 tokens: the token-by-token kernel (default) and the
+    chunked path (short-call threshold 0) both match the oracle, state in and
+    out, bf16 output included."""
+    B, H = 2, 3
+    inp = inputs.generate(B, T, H, dk, dv, dtype, seed=3000 + T + dk + dv)
+    s0 = _state(B, H, dk, dv, seed=T + 7)
+    d = to_dev(inp)
+    prev = gdn.gdn_set_short_call_tokens(64 if path == "token" else 0)
+    gdn.gdn_set_kernel_timing(1)
+    gdn.gdn_read_kernel_timing()
+    try:
+        o, s = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"], s0.cuda())
+        o16, _ = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"], s0.cuda(),
+                                 out_dtype=torch.bfloat16)
+        names = set(gdn.gdn_read_kernel_timing())
+    finally:
+        gdn.gdn_set_kernel_timing(0)
+        gdn.gdn_set_short_call_tokens(prev)
+    assert (names == {"token_step"}) == (path == "token"), names
+    o_ref, s_ref = oracle_heads(inp, state_in=s0)
+    tol = TOL[DT[dtype]]
+    assert rel_err(o, o_ref) <= tol
+    assert rel_err(s, s_ref) <= tol
+    assert rel_err_bf16_out(o16, o_ref) <= TOL[torch.bfloat16]
+
+
+def test_short_call_threshold_switches_path():
+    """A 65-token call takes the chunked path whatever the threshold (it is
+    clamped to 64); a 64-token call takes the token path by default."""
+    inp = inputs.generate(1, 65, 2, 128, 128, "bf16", seed=5)
+    d = to_dev(inp)
+    gdn.gdn_set_kernel_timing(1)
+    gdn.gdn_read_kernel_timing()
+    try:
+        prev = gdn.gdn_set_short_call_tokens(1000)
+        gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+        gdn.scan_causal(d["q"][:, :64].contiguous(), d["k"][:, :64].contiguous(), d["v"][:, :64].contiguous(),
+                        d["alpha"][:, :64].contiguous(), d["beta"][:, :64].contiguous())
+        names = set(gdn.gdn_read_kernel_timing())
+    finally:
+        gdn.gdn_set_kernel_timing(0)
+        gdn.gdn_set_short_call_tokens(prev)
+    assert "token_step" in names
+    assert names - {"token_step"}, names
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (128, 64)])
 @pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 130, 257])
@@ -217,3 +268,39 @@ def test_many_heads_take_wide_slices(mode, o_dtype):
         assert rel_err_bf16_out(o, o_ref) <= TOL[torch.bfloat16]
     if mode == "causal":
         assert rel_err(s, s_ref) <= TOL[torch.bfloat16]
+
+
+def test_rollout_replays_in_a_cuda_graph():
+    """A rollout of gdn_step calls (chunked and token-by-token ones) captured in
+    one CUDA graph replays to the same bits as the eager calls."""
+    B, H, dk, dv = 1, 4, 128, 128
+    lens = [200, 40, 1, 130, 64, 65]
+    T = sum(lens)
+    inp = inputs.generate(B, T, H, dk, dv, "bf16", seed=91)
+    d = to_dev(inp)
+    cuts = np.concatenate([[0], np.cumsum(lens)])
+    ws = torch.empty(gdn.workspace_size(B, max(lens), H, dk, dv, torch.bfloat16), dtype=torch.uint8,
+                     device="cuda")
+
+    def rollout(state, o):
+        state.zero_()
+        for a, b in zip(cuts, cuts[1:]):
+            sl = {n: t[:, a:b] for n, t in d.items()}
+            gdn.step(sl["q"], sl["k"], sl["v"], sl["alpha"], sl["beta"], state, out=o[:, a:b], workspace=ws)
+
+    s_e = torch.empty(B, H, dk, dv, device="cuda")
+    o_e = torch.empty(B, T, H, dv, device="cuda")
+    rollout(s_e, o_e)                      # eager (also the warm-up before capture)
+    torch.cuda.synchronize()
+    s_g = torch.empty_like(s_e)
+    o_g = torch.full_like(o_e, float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        rollout(s_g, o_g)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o_g, o_e)
+    assert torch.equal(s_g, s_e)
+    o_ref, s_ref = oracle_heads(inp)
+    assert rel_err(o_g, o_ref) <= TOL[torch.bfloat16]
+    assert rel_err(s_g, s_ref) <= TOL[torch.bfloat16]
