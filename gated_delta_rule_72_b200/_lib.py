@@ -23,6 +23,8 @@ _P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 SIGNATURES = {
     "gdn_scan_causal": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "gdn_scan_bidir": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
+    "gdn_scan_bidir_states": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                   _P, _Z, _P]),
     "gdn_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "gdn_step_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "gdn_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
@@ -72,6 +74,13 @@ def gdn_scan_bidir(q, k, v, alpha, beta, o, B, T, H, dk, dv, dt, o_dt, workspace
                    stream):
     return load().gdn_scan_bidir(q, k, v, alpha, beta, o, B, T, H, dk, dv, dt, o_dt, workspace,
                                  ws_bytes, stream)
+
+
+def gdn_scan_bidir_states(q, k, v, alpha, beta, state_in, state_in_bwd, state_out, state_out_bwd, o,
+                          B, T, H, dk, dv, dt, o_dt, workspace, ws_bytes, stream):
+    return load().gdn_scan_bidir_states(q, k, v, alpha, beta, state_in, state_in_bwd, state_out,
+                                        state_out_bwd, o, B, T, H, dk, dv, dt, o_dt, workspace,
+                                        ws_bytes, stream)
 
 
 def gdn_step(q, k, v, alpha, beta, state, o, B, T, H, dk, dv, dt, o_dt, workspace, ws_bytes,

@@ -91,17 +91,35 @@ def scan_causal(q, k, v, alpha, beta, state=None, *, return_state=True, out=None
     return o, state_out
 
 
-def scan_bidir(q, k, v, alpha, beta, *, out=None, out_dtype=torch.float32, workspace=None):
-    """Bidirectional scan (causal + strict reverse readouts, summed in fp32)."""
+def scan_bidir(q, k, v, alpha, beta, *, out=None, out_dtype=torch.float32, workspace=None,
+               state=None, state_bwd=None, return_states=False):
+    """Bidirectional scan (causal + strict reverse readouts, summed in fp32).
+
+    state / state_bwd: initial states ([B,H,dk,dv] fp32) of the causal scan
+    (S_0) and of the reverse scan (R_{T+1}); None = zero.  Returns o, or with
+    return_states=True (o, S_T, R_1)."""
     B, T, H, dk, dv, dt = _dims(q, k, v, alpha, beta)
+    for t, name in ((state, "state"), (state_bwd, "state_bwd")):
+        if t is not None:
+            _check(t, name, torch.float32, (B, H, dk, dv))
     o, odt = _out(B, T, H, dv, q.device, out, out_dtype)
     ws, nbytes = _workspace(workspace_size(B, T, H, dk, dv, q.dtype, True, o.dtype), q.device,
                             workspace)
     stream = torch.cuda.current_stream(q.device).cuda_stream
-    st = _lib.gdn_scan_bidir(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
-                             B, T, H, dk, dv, dt, odt, _ptr(ws), nbytes, stream)
-    _raise("gdn_scan_bidir", st)
-    return o
+    if state is None and state_bwd is None and not return_states:
+        st = _lib.gdn_scan_bidir(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
+                                 B, T, H, dk, dv, dt, odt, _ptr(ws), nbytes, stream)
+        _raise("gdn_scan_bidir", st)
+        return o
+    s_out = s_out_b = None
+    if return_states:
+        s_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+        s_out_b = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = _lib.gdn_scan_bidir_states(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state),
+                                    _ptr(state_bwd), _ptr(s_out), _ptr(s_out_b), _ptr(o), B, T, H, dk,
+                                    dv, dt, odt, _ptr(ws), nbytes, stream)
+    _raise("gdn_scan_bidir_states", st)
+    return (o, s_out, s_out_b) if return_states else o
 
 
 def step(q, k, v, alpha, beta, state, *, out=None, out_dtype=torch.float32, workspace=None):

@@ -37,6 +37,9 @@ struct Args {
     void *ws;
     size_t ws_bytes;
     cudaStream_t stream;
+    // bidirectional calls: the reverse direction's initial R_{T+1} and final R_1
+    const float *state_in_bwd = nullptr;
+    float *state_out_bwd = nullptr;
 };
 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -74,13 +77,21 @@ gdn_status check_common(const Args &a, bool need_inputs) {
         // the gates are read one float at a time
         if (!aligned(a.alpha, 4) || !aligned(a.beta, 4)) return GDN_ERR_ALIGN;
     }
-    if (a.state_in && !aligned(a.state_in, 16)) return GDN_ERR_ALIGN;
-    if (a.state_out && !aligned(a.state_out, 16)) return GDN_ERR_ALIGN;
-    if (a.state_in && a.state_out && a.state_in != a.state_out) {
-        const size_t n = (size_t)a.B * a.H * a.dk * a.dv * sizeof(float);
-        const char *i0 = (const char *)a.state_in, *o0 = (const char *)a.state_out;
-        if (i0 < o0 + n && o0 < i0 + n) return GDN_ERR_SHAPE;  // partial overlap
-    }
+    const void *st[4] = {a.state_in, a.state_out, a.state_in_bwd, a.state_out_bwd};
+    for (const void *p : st)
+        if (p && !aligned(p, 16)) return GDN_ERR_ALIGN;
+    // An output state may be its own direction's input state exactly; no other
+    // two of the four state buffers may overlap.
+    const size_t n = (size_t)a.B * a.H * a.dk * a.dv * sizeof(float);
+    auto overlap = [n](const void *x, const void *y) {
+        const char *p = static_cast<const char *>(x), *q = static_cast<const char *>(y);
+        return p && q && p < q + n && q < p + n;
+    };
+    for (int i = 0; i < 4; ++i)
+        for (int j = i + 1; j < 4; ++j) {
+            const bool own = (i == 0 && j == 1) || (i == 2 && j == 3);
+            if (overlap(st[i], st[j]) && !(own && st[i] == st[j])) return GDN_ERR_SHAPE;
+        }
     return GDN_OK;
 }
 
@@ -97,13 +108,19 @@ gdn_status launch_status() {
 }
 
 // T = 0: state_out <- state_in (or zero).
-gdn_status empty_scan(const Args &a) {
-    if (!a.state_out || a.state_out == a.state_in) return GDN_OK;
+gdn_status copy_state(const Args &a, const float *in, float *out) {
+    if (!out || out == in) return GDN_OK;
     const size_t n = (size_t)a.B * a.H * a.dk * a.dv * sizeof(float);
-    cudaError_t e = a.state_in
-        ? cudaMemcpyAsync(a.state_out, a.state_in, n, cudaMemcpyDeviceToDevice, a.stream)
-        : cudaMemsetAsync(a.state_out, 0, n, a.stream);
+    cudaError_t e = in ? cudaMemcpyAsync(out, in, n, cudaMemcpyDeviceToDevice, a.stream)
+                       : cudaMemsetAsync(out, 0, n, a.stream);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// T = 0: every final state is its initial state (zero if none).
+gdn_status empty_scan(const Args &a, int bidir) {
+    const gdn_status s = copy_state(a, a.state_in, a.state_out);
+    if (s != GDN_OK || !bidir) return s;
+    return copy_state(a, a.state_in_bwd, a.state_out_bwd);
 }
 
 // ---------------------------------------------------------------------------
@@ -146,12 +163,12 @@ gdn_status run_simt(const Args &a, int bidir) {
     }
     {
         gdn::LaunchScope ls("simt_chain", a.stream);
-        chain<<<grid, 256, chain_smem, a.stream>>>(rec, nullptr, nullptr, o, part, a.T, a.H, nC,
+        chain<<<grid, 256, chain_smem, a.stream>>>(rec, a.state_in, a.state_out, o, part, a.T, a.H, nC,
                                                    0, kOutPartial, nbh);
     }
     if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
     gdn::LaunchScope ls("simt_chain", a.stream);
-    chain<<<grid, 256, chain_smem, a.stream>>>(rec, nullptr, nullptr, o, part, a.T, a.H, nC, 1,
+    chain<<<grid, 256, chain_smem, a.stream>>>(rec, a.state_in_bwd, a.state_out_bwd, o, part, a.T, a.H, nC, 1,
                                                kOutAddPartial, nbh);
     return launch_status();
 }
@@ -306,8 +323,8 @@ __global__ void cast_bf16_kernel(const float4 *__restrict__ sum, uint2 *__restri
 // (kOutPair, both directions adding up there).
 template <int DV, int NS, typename Tout>
 gdn_status launch_chain(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq,
-                        const unsigned char *recs, int nC, int ndir, const float *state_in,
-                        float *state_out, const gdn::tc2::ChainOut<Tout> &out, const void *target,
+                        const unsigned char *recs, int nC, int ndir, const gdn::tc2::ChainStates &states,
+                        const gdn::tc2::ChainOut<Tout> &out, const void *target,
                         unsigned int *err) {
     using SM = gdn::tc2::ChainSmem<NS>;
     const bool f32t = std::is_same<Tout, float>::value || out.mode == gdn::tc2::kOutPair;
@@ -319,18 +336,18 @@ gdn_status launch_chain(const Args &a, const CUtensorMap &mk, const CUtensorMap 
         return GDN_ERR_CUDA;
     gdn::LaunchScope ls(ndir == 2 ? "tc_chain_bidir" : "tc_chain", a.stream);
     kern<<<dim3(DV / NS, a.B * a.H, ndir), gdn::tc2::chain_threads<NS>(), SM::kAlloc, a.stream>>>(
-        mk, mq, mo, recs, state_in, state_out, out, a.T, a.H, nC, err);
+        mk, mq, mo, recs, states, out, a.T, a.H, nC, err);
     return launch_status();
 }
 
 template <int DV, typename Tout>
 gdn_status launch_chain_ns(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq,
-                           const unsigned char *recs, int nC, int ndir, const float *state_in,
-                           float *state_out, const gdn::tc2::ChainOut<Tout> &out, const void *target,
+                           const unsigned char *recs, int nC, int ndir, const gdn::tc2::ChainStates &states,
+                           const gdn::tc2::ChainOut<Tout> &out, const void *target,
                            unsigned int *err) {
     if (chain_slice_cols(a.B, a.H, DV, ndir) == 32)
-        return launch_chain<DV, 32, Tout>(a, mk, mq, recs, nC, ndir, state_in, state_out, out, target, err);
-    return launch_chain<DV, 64, Tout>(a, mk, mq, recs, nC, ndir, state_in, state_out, out, target, err);
+        return launch_chain<DV, 32, Tout>(a, mk, mq, recs, nC, ndir, states, out, target, err);
+    return launch_chain<DV, 64, Tout>(a, mk, mq, recs, nC, ndir, states, out, target, err);
 }
 
 // Prep and chain in one cooperative launch (tc_fused.cuh): n_chain chain CTAs
@@ -339,7 +356,7 @@ gdn_status launch_chain_ns(const Args &a, const CUtensorMap &mk, const CUtensorM
 template <int DV, int NS, typename Tout>
 gdn_status launch_fused(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq, const CUtensorMap &mv,
                         unsigned char *recs, unsigned int *ready, int nC, int ndir, int n_chain, int n_prep,
-                        const float *state_in, float *state_out, const gdn::tc2::ChainOut<Tout> &out,
+                        const gdn::tc2::ChainStates &states, const gdn::tc2::ChainOut<Tout> &out,
                         const void *target, unsigned int *err) {
     const bool f32t = std::is_same<Tout, float>::value || out.mode == gdn::tc2::kOutPair;
     CUtensorMap mo;
@@ -366,8 +383,8 @@ gdn_status launch_fused(const Args &a, const CUtensorMap &mk, const CUtensorMap 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     gdn::LaunchScope ls("tc_fused", a.stream);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, mo, a.alpha, a.beta, recs, ready, state_in,
-                                             state_out, out, a.T, a.H, nC, a.B * a.H, ndir, n_chain, err);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, mo, a.alpha, a.beta, recs, ready, states,
+                                             out, a.T, a.H, nC, a.B * a.H, ndir, n_chain, err);
     if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorNotSupported) {
         (void)cudaGetLastError();
         return GDN_ERR_UNSUPPORTED;
@@ -415,8 +432,13 @@ gdn_status run_tc(const Args &a, int bidir) {
     } else {
         out.mode = gdn::tc2::kOutStore;
     }
-    const float *s_in = bidir ? nullptr : a.state_in;
-    float *s_out = bidir ? nullptr : a.state_out;
+    gdn::tc2::ChainStates states{};
+    states.in[0] = a.state_in;
+    states.out[0] = a.state_out;
+    if (bidir) {
+        states.in[1] = a.state_in_bwd;
+        states.out[1] = a.state_out_bwd;
+    }
 
     // One cooperative launch (prep on the SMs the chain leaves free) when the
     // chain grid leaves room for it; else prep, then chain.
@@ -428,15 +450,15 @@ gdn_status run_tc(const Args &a, int bidir) {
         if (cudaMemsetAsync(ready, 0, (size_t)ndir * a.B * a.H * nC * sizeof(unsigned int), a.stream) != cudaSuccess)
             return GDN_ERR_CUDA;
         const int n_prep = sms - (int)n_chain;
-        s = ns == 32 ? launch_fused<DV, 32, Tout>(a, mk, mq, mv, recs, ready, nC, ndir, (int)n_chain, n_prep, s_in,
-                                                  s_out, out, target, err)
-                     : launch_fused<DV, 64, Tout>(a, mk, mq, mv, recs, ready, nC, ndir, (int)n_chain, n_prep, s_in,
-                                                  s_out, out, target, err);
+        s = ns == 32 ? launch_fused<DV, 32, Tout>(a, mk, mq, mv, recs, ready, nC, ndir, (int)n_chain, n_prep, states,
+                                                  out, target, err)
+                     : launch_fused<DV, 64, Tout>(a, mk, mq, mv, recs, ready, nC, ndir, (int)n_chain, n_prep, states,
+                                                  out, target, err);
     }
     if (s == GDN_ERR_UNSUPPORTED) {
         s = launch_prep<DV>(a, mk, mq, mv, recs, nC, ndir, err);
         if (s != GDN_OK) return s;
-        s = launch_chain_ns<DV, Tout>(a, mk, mq, recs, nC, ndir, s_in, s_out, out, target, err);
+        s = launch_chain_ns<DV, Tout>(a, mk, mq, recs, nC, ndir, states, out, target, err);
     }
     if (s != GDN_OK || !bidir || f32_out) return s;
     gdn::LaunchScope ls("tc_bidir_cast", a.stream);
@@ -502,7 +524,7 @@ gdn_status run(const Args &a, int bidir) {
     const gdn_status s =
         check_ws(a, plan_workspace(a.B, a.T, a.H, a.dk, a.dv, a.dt, a.o_dt, bidir));
     if (s != GDN_OK) return s;
-    if (a.T == 0) return bidir ? GDN_OK : empty_scan(a);
+    if (a.T == 0) return empty_scan(a, bidir);
     if (!bidir && take_token_path(a)) return run_short(a);
     if (use_tc(a.dt, a.dk, a.dv)) return dispatch_tc(a, bidir);
     return a.dt == GDN_F32 ? dispatch_out<float>(a, bidir) : dispatch_out<__nv_bfloat16>(a, bidir);
@@ -561,6 +583,18 @@ gdn_status gdn_scan_bidir(const void *q, const void *k, const void *v, const flo
                           void *stream) {
     Args a{q, k, v, alpha, beta, nullptr, nullptr, o, B, T, H, dk, dv, dt, o_dt,
            workspace, ws_bytes, static_cast<cudaStream_t>(stream)};
+    gdn_status s = check_common(a, T > 0);
+    if (s != GDN_OK) return s;
+    return run(a, 1);
+}
+
+gdn_status gdn_scan_bidir_states(const void *q, const void *k, const void *v, const float *alpha,
+                                 const float *beta, const float *state_in, const float *state_in_bwd,
+                                 float *state_out, float *state_out_bwd, void *o, int B, int T, int H,
+                                 int dk, int dv, gdn_dtype dt, gdn_dtype o_dt, void *workspace,
+                                 size_t ws_bytes, void *stream) {
+    Args a{q, k, v, alpha, beta, state_in, state_out, o, B, T, H, dk, dv, dt, o_dt,
+           workspace, ws_bytes, static_cast<cudaStream_t>(stream), state_in_bwd, state_out_bwd};
     gdn_status s = check_common(a, T > 0);
     if (s != GDN_OK) return s;
     return run(a, 1);

@@ -107,6 +107,13 @@ __host__ __device__ constexpr int chain_threads() { return 21 * 32; }
 
 enum OutMode { kOutStore = 0, kOutPair = 1 };
 
+// Initial and final states per direction ([B, H, d_k, d_v] fp32 each; null:
+// zero / not written).  Direction 0 is the causal scan, 1 the reverse one.
+struct ChainStates {
+    const float *in[2];
+    float *out[2];
+};
+
 template <typename Tout>
 __device__ __forceinline__ void store4(Tout *p, float4 v);
 template <>
@@ -162,7 +169,7 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float *v) {
 template <int DV, int NS, typename Tout>
 __device__ __forceinline__ void chain_body(
     const CUtensorMap *tm_k, const CUtensorMap *tm_q, const CUtensorMap *tm_o,
-    const unsigned char *__restrict__ recs, const float *__restrict__ state_in, float *__restrict__ state_out,
+    const unsigned char *__restrict__ recs, const ChainStates &states,
     const ChainOut<Tout> &out, const unsigned int *__restrict__ ready, int T, int H, int nC, int slice,
     int bh, int dir, int nslices, int nbh, unsigned char *smem, unsigned int *__restrict__ err)
 {
@@ -235,6 +242,7 @@ __device__ __forceinline__ void chain_body(
     auto de_off = [&](int n, int k) { return (N2 > 64 ? (n >> 6) * SM::kGrpDE : 0) + swz128(k * 128 + (n & 63) * 2); };
     float S[NC];
     if (warp < 16) {
+        const float *state_in = dir ? states.in[1] : states.in[0];   // (a select: no local copy)
         const float *src = state_in ? state_in + ((size_t)bh * kDK + d_row) * DV + j0 + n0 : nullptr;
 #pragma unroll
         for (int n = 0; n < NC; ++n) S[n] = src ? src[n] : 0.f;
@@ -614,6 +622,7 @@ __device__ __forceinline__ void chain_body(
             }
             if (tid == 0) CHAIN_TS(19);
         }
+        float *state_out = dir ? states.out[1] : states.out[0];
         if (!*abort_s && state_out) {
             float *dst = state_out + ((size_t)bh * kDK + d_row) * DV + j0 + n0;
 #pragma unroll
@@ -643,12 +652,12 @@ template <int DV, int NS, typename Tout>
 __global__ void __launch_bounds__(chain_threads<NS>(), 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
              const __grid_constant__ CUtensorMap tm_o, const unsigned char *__restrict__ recs,
-             const float *__restrict__ state_in, float *__restrict__ state_out, const ChainOut<Tout> out,
+             const ChainStates states, const ChainOut<Tout> out,
              int T, int H, int nC, unsigned int *__restrict__ err)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    chain_body<DV, NS, Tout>(&tm_k, &tm_q, &tm_o, recs, state_in, state_out, out, nullptr, T, H, nC, blockIdx.x,
+    chain_body<DV, NS, Tout>(&tm_k, &tm_q, &tm_o, recs, states, out, nullptr, T, H, nC, blockIdx.x,
                              blockIdx.y, blockIdx.z, gridDim.x, gridDim.y, smem, err);
 }
 

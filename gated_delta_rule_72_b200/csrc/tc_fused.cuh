@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(chain_threads<NS>(), 1)
 fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
              const float *__restrict__ alpha, const float *__restrict__ beta, unsigned char *__restrict__ recs,
-             unsigned int *__restrict__ ready, const float *__restrict__ state_in, float *__restrict__ state_out,
+             unsigned int *__restrict__ ready, const ChainStates states,
              const ChainOut<Tout> out, int T, int H, int nC, int nbh, int ndir, int n_chain,
              unsigned int *__restrict__ err)
 {
@@ -50,7 +50,7 @@ fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     const int nsl = DV / NS;
     if ((int)blockIdx.x < n_chain) {
         const int i = blockIdx.x;
-        chain_body<DV, NS, Tout>(&tm_k, &tm_q, &tm_o, recs, state_in, state_out, out, ready, T, H, nC, i % nsl,
+        chain_body<DV, NS, Tout>(&tm_k, &tm_q, &tm_o, recs, states, out, ready, T, H, nC, i % nsl,
                                  (i / nsl) % nbh, i / (nsl * nbh), nsl, nbh, smem, err);
         return;
     }

@@ -104,6 +104,31 @@ GDN_API gdn_status gdn_scan_bidir(const void *q, const void *k, const void *v,
                           void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * gdn_scan_bidir_states -- gdn_scan_bidir with an initial and a final state
+ * per direction (for instance a conditioning context folded into the states
+ * a clip's two scans start from):
+ *   causal half   S_0 = state_in (NULL: zero), S_t as in gdn_scan_causal;
+ *                 state_out (NULL: not written) <- S_T
+ *   reverse half  R_{T+1} = state_in_bwd (NULL: zero),
+ *                 R_t = alpha_t (I - beta_t k_t k_t^T) R_{t+1} + beta_t k_t v_t^T;
+ *                 state_out_bwd (NULL: not written) <- R_1
+ *   o_t = S_t^T q_t + R_{t+1}^T q_t
+ * Each state is [B, H, dk, dv] fp32, 16-byte aligned.  An output state may
+ * be its own direction's input state (updated in place); no other two of the
+ * four may overlap (GDN_ERR_SHAPE).  With T = 0 each output state receives
+ * its input state.  Workspace: gdn_workspace_size(..., bidir = 1).  Sources:
+ * as gdn_scan_bidir; the initial states of the two scans are the
+ * bidirectional form's counterpart of the causal scan's state in and out.
+ */
+GDN_API gdn_status gdn_scan_bidir_states(const void *q, const void *k, const void *v,
+                                         const float *alpha, const float *beta,
+                                         const float *state_in, const float *state_in_bwd,
+                                         float *state_out, float *state_out_bwd, void *o,
+                                         int B, int T, int H, int dk, int dv, gdn_dtype dt,
+                                         gdn_dtype o_dt, void *workspace, size_t ws_bytes,
+                                         void *stream);
+
+/*
  * gdn_step -- one streaming call: gdn_scan_causal with state_in == state_out
  * == state (required, updated in place).  A rollout is a sequence of
  * gdn_step calls on successive slices of the token stream; the result equals

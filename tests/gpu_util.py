@@ -30,9 +30,11 @@ def rel_err_bf16_out(x, ref) -> float:
     return float(max(np.max(excess), 0.0) / rms)
 
 
-def oracle_heads(inp, heads=None, mode="causal", state_in=None, t_slice=None):
+def oracle_heads(inp, heads=None, mode="causal", state_in=None, t_slice=None, state_in_bwd=None,
+                 with_bwd=False):
     """Oracle on a subset of heads (all if None); inputs are the CPU copies of
-    exactly the tensors the GPU used.  Returns numpy (o, state_out)."""
+    exactly the tensors the GPU used.  Returns numpy (o, state_out), or with
+    with_bwd (o, state_out, reverse state_out)."""
     def pick(t, axis_h):
         t = t.detach().cpu()
         if t_slice is not None and axis_h == 2:
@@ -43,8 +45,9 @@ def oracle_heads(inp, heads=None, mode="causal", state_in=None, t_slice=None):
     q, k, v = (pick(inp[n], 2) for n in ("q", "k", "v"))
     a, b = pick(inp["alpha"], 2), pick(inp["beta"], 2)
     s0 = None if state_in is None else pick(state_in, 1)
-    o, sf, _ = oracle.scan(q, k, v, a, b, mode=mode, state_in=s0)
-    return o, sf
+    r0 = None if state_in_bwd is None else pick(state_in_bwd, 1)
+    o, sf, sb = oracle.scan(q, k, v, a, b, mode=mode, state_in=s0, state_in_bwd=r0)
+    return (o, sf, sb) if with_bwd else (o, sf)
 
 
 def to_dev(inp, device="cuda"):

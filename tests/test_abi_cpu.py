@@ -154,3 +154,27 @@ def test_short_call_threshold_is_clamped(lib):
         assert lib.gdn_set_short_call_tokens(17) == 17
     finally:
         lib.gdn_set_short_call_tokens(prev)
+
+
+def _bidir_states(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, alpha=FAKE, beta=FAKE, state_in=None, state_in_bwd=None,
+             state_out=None, state_out_bwd=None, o=FAKE, B=1, T=64, H=2, dk=64, dv=64, dt=0, o_dt=0,
+             workspace=FAKE, ws_bytes=10, stream=None)
+    a.update(kw)
+    return _lib.gdn_scan_bidir_states(*a.values())
+
+
+def test_bidir_states_rejects_before_launch(lib):
+    """Overlap and alignment rules of the four state buffers, checked before
+    the workspace size (ws_bytes=10 would otherwise give -6)."""
+    S = 1 << 16                      # bytes of one state: 1*2*64*64*4 = 32 KB < 64 KB apart
+    A, Bb, C, D = FAKE, FAKE + S, FAKE + 2 * S, FAKE + 3 * S
+    assert _bidir_states(state_in=A + 4) == -4
+    assert _bidir_states(state_out_bwd=D + 8) == -4
+    # both outputs in one buffer, or an output over the other direction's input
+    assert _bidir_states(state_out=C, state_out_bwd=C) == -2
+    assert _bidir_states(state_in=A, state_out_bwd=A) == -2
+    assert _bidir_states(state_in_bwd=Bb, state_out=Bb + 256) == -2
+    # each direction in place, or four separate buffers: only the workspace is short
+    assert _bidir_states(state_in=A, state_out=A, state_in_bwd=Bb, state_out_bwd=Bb) == -6
+    assert _bidir_states(state_in=A, state_in_bwd=Bb, state_out=C, state_out_bwd=D) == -6

@@ -260,6 +260,34 @@ def test_reverse_equals_causal_on_reversed_suffix():
     np.testing.assert_allclose(R1, S_all, rtol=1e-12, atol=1e-13)
 
 
+def test_bidir_with_initial_states_in_both_directions():
+    """Bidirectional with a causal initial state S_0 and a reverse initial
+    state R_{T+1}: the reverse readout at t is q_t read against a causal run
+    over the time-reversed suffix x_T .. x_{t+1} started from R_{T+1}; the
+    causal half is the causal scan from S_0; the two add up; the final reverse
+    state R_1 is the causal state of the whole reversed sequence from R_{T+1}."""
+    rng = np.random.default_rng(14)
+    T, H, dk, dv = 9, 2, 4, 3
+    q, k, v, a, b = _rand(rng, 1, T, H, dk, dv)
+    S0 = rng.normal(size=(1, H, dk, dv))
+    R0 = rng.normal(size=(1, H, dk, dv))
+    o, sf, sb = oracle.scan(q, k, v, a, b, mode="bidir", state_in=S0, state_in_bwd=R0)
+    o_c, s_c, _ = oracle.scan(q, k, v, a, b, state_in=S0)
+    rev = lambda x: x[:, ::-1]
+    for t in range(T):
+        suf = slice(t + 1, T)
+        if t + 1 < T:
+            _, S, _ = oracle.scan(rev(q[:, suf]), rev(k[:, suf]), rev(v[:, suf]),
+                                  rev(a[:, suf]), rev(b[:, suf]), state_in=R0)
+        else:
+            S = R0
+        want = o_c[0, t] + np.einsum("hij,hi->hj", S[0], q[0, t])
+        np.testing.assert_allclose(o[0, t], want, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sf, s_c, rtol=1e-12, atol=1e-13)
+    _, S_all, _ = oracle.scan(rev(q), rev(k), rev(v), rev(a), rev(b), state_in=R0)
+    np.testing.assert_allclose(sb, S_all, rtol=1e-12, atol=1e-13)
+
+
 # --------------------------------------------------------------------------
 # streaming: state in / state out
 # --------------------------------------------------------------------------

@@ -115,6 +115,58 @@ def test_bidir_shapes(dtype, dk, dv, T):
     assert rel_err(o, o_ref) <= TOL[DT[dtype]]
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (128, 64)])
+@pytest.mark.parametrize("T", [1, 64, 130])
+def test_bidir_initial_states(dtype, dk, dv, T):
+    """Bidirectional with a causal initial state S_0 and a reverse initial
+    state R_{T+1}: o and both final states (S_T, R_1) against the oracle."""
+    B, H = 1, 3
+    inp = inputs.generate(B, T, H, dk, dv, dtype, seed=2500 + T + dk + dv)
+    s0, r0 = _state(B, H, dk, dv, seed=T + 1), _state(B, H, dk, dv, seed=T + 2)
+    d = to_dev(inp)
+    o, sf, sb = gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"], state=s0.cuda(),
+                               state_bwd=r0.cuda(), return_states=True)
+    torch.cuda.synchronize()
+    o_ref, sf_ref, sb_ref = oracle_heads(inp, mode="bidir", state_in=s0, state_in_bwd=r0, with_bwd=True)
+    tol = TOL[DT[dtype]]
+    assert rel_err(o, o_ref) <= tol
+    assert rel_err(sf, sf_ref) <= tol
+    assert rel_err(sb, sb_ref) <= tol
+
+
+@pytest.mark.parametrize("H", [3, 40])
+def test_bidir_states_in_place(H):
+    """Output states updated in place (each direction's buffer holds its
+    initial state, then its final one), on the fused launch (H = 3) and the
+    two-launch path with 64-column slices (H = 40); T = 0 passes the states
+    through."""
+    B, T, dk, dv = 1, 130, 128, 128
+    inp = inputs.generate(B, T, H, dk, dv, "bf16", seed=2600 + H)
+    s0, r0 = _state(B, H, dk, dv, seed=H), _state(B, H, dk, dv, seed=H + 50)
+    d = to_dev(inp)
+    sf, sb = s0.cuda(), r0.cuda()
+    B_, T_, H_, dk_, dv_ = B, T, H, dk, dv
+    o = torch.empty(B, T, H, dv, device="cuda")
+    ws = torch.empty(gdn.workspace_size(B, T, H, dk, dv, torch.bfloat16, bidir=True), dtype=torch.uint8,
+                     device="cuda")
+    st = gdn.gdn_scan_bidir_states(d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(),
+                                   d["alpha"].data_ptr(), d["beta"].data_ptr(), sf.data_ptr(), sb.data_ptr(),
+                                   sf.data_ptr(), sb.data_ptr(), o.data_ptr(), B_, T_, H_, dk_, dv_, 1, 0,
+                                   ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    torch.cuda.synchronize()
+    o_ref, sf_ref, sb_ref = oracle_heads(inp, mode="bidir", state_in=s0, state_in_bwd=r0, with_bwd=True)
+    assert rel_err(o, o_ref) <= TOL[torch.bfloat16]
+    assert rel_err(sf, sf_ref) <= TOL[torch.bfloat16]
+    assert rel_err(sb, sb_ref) <= TOL[torch.bfloat16]
+    e = {n: t[:, :0].contiguous() for n, t in d.items()}
+    o0, sf0, sb0 = gdn.scan_bidir(e["q"], e["k"], e["v"], e["alpha"], e["beta"], state=sf, state_bwd=sb,
+                                  return_states=True)
+    torch.cuda.synchronize()
+    assert torch.equal(sf0, sf) and torch.equal(sb0, sb)
+
+
 @pytest.mark.parametrize("gates", ["default", "skewed"])
 def test_streaming_splits_match_one_call(gates):
     """gdn_step over arbitrary call boundaries (lengths 1, 63, 64, 65, ...)
