@@ -89,3 +89,33 @@ def scan(q, k, v, alpha, beta, mode="causal", state_in=None, state_in_bwd=None,
     if rc != 0:
         raise RuntimeError("gdn_oracle_scan failed (%d)" % rc)
     return o, sf, sb
+
+
+def readout_gate(o, z, gamma=None, eps=1e-6):
+    """Readout epilogue of the linear branch, in float64: per (b, t, h) row of
+    d_v values, the RMS-normalised readout scaled per channel by gamma and by
+    the sigmoid of the content-dependent gate z:
+
+        y = o / sqrt(mean(o ** 2) + eps) * gamma * 1 / (1 + exp(-z))
+
+    Source: AI summary of "Video DeltaNet: A Video-Native Hybrid Attention for
+    Livestream Video Generation", "Key Contributions" 1 (each branch has its
+    own content-dependent sigmoid gate; the linear branch's readout is RMS
+    normalised).  The page fixes neither the axis nor the order; the reading
+    taken here: the norm runs over the head's d_v channels of one token, and
+    the gate multiplies the normalised readout.  gamma None = ones.
+    o, z: [B, T, H, dv]; gamma: [dv].  Returns float64 [B, T, H, dv]."""
+    o = _f64(o)
+    z = _f64(z)
+    assert o.shape == z.shape
+    dv = o.shape[-1]
+    g = np.ones(dv) if gamma is None else _f64(gamma)
+    assert g.shape == (dv,)
+    y = np.empty_like(o)
+    flat_o, flat_z, flat_y = o.reshape(-1, dv), z.reshape(-1, dv), y.reshape(-1, dv)
+    for r in range(flat_o.shape[0]):
+        row = flat_o[r]
+        inv = 1.0 / np.sqrt(np.mean(row * row) + eps)
+        for j in range(dv):
+            flat_y[r, j] = row[j] * inv * g[j] / (1.0 + np.exp(-flat_z[r, j]))
+    return y

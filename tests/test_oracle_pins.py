@@ -322,3 +322,31 @@ def test_threads_do_not_change_results():
     o1, s1, _ = oracle.scan(q, k, v, a, b, mode="bidir", threads=1)
     o2, s2, _ = oracle.scan(q, k, v, a, b, mode="bidir", threads=7)
     np.testing.assert_array_equal(o1, o2)
+
+
+# --------------------------------------------------------------------------
+# readout epilogue: RMS norm over d_v, per-channel gain, sigmoid gate
+# --------------------------------------------------------------------------
+def test_readout_worked_example():
+    """o = (3, 4): mean of squares 12.5; gate z = (0, ln 3) gives sigmoid
+    (1/2, 3/4); gain (2, 1): both outputs equal 3 / sqrt(12.5)."""
+    o = np.array([3.0, 4.0]).reshape(1, 1, 1, 2)
+    z = np.array([0.0, np.log(3.0)]).reshape(1, 1, 1, 2)
+    y = oracle.readout_gate(o, z, gamma=np.array([2.0, 1.0]), eps=0.0)
+    np.testing.assert_allclose(y.ravel(), [3 / np.sqrt(12.5)] * 2, rtol=1e-15)
+
+
+def test_readout_normalises_and_gates():
+    rng = np.random.default_rng(21)
+    o = rng.normal(size=(2, 5, 3, 8)) * rng.uniform(0.1, 10, size=(2, 5, 3, 1))
+    open_gate = np.full(o.shape, 40.0)         # sigmoid(40) = 1 in float64
+    y = oracle.readout_gate(o, open_gate, eps=0.0)
+    np.testing.assert_allclose(np.mean(y * y, axis=-1), 1.0, rtol=1e-14)     # unit RMS per row
+    np.testing.assert_allclose(oracle.readout_gate(7.5 * o, open_gate, eps=0.0), y, rtol=1e-14)
+    np.testing.assert_allclose(oracle.readout_gate(o, np.zeros(o.shape), eps=0.0), 0.5 * y, rtol=1e-14)
+    g = rng.uniform(0.5, 2.0, size=8)
+    np.testing.assert_allclose(oracle.readout_gate(o, open_gate, gamma=g, eps=0.0), y * g, rtol=1e-14)
+    # eps adds to the mean of squares: a row of zeros stays zero, a constant row c gives c / sqrt(c^2 + eps)
+    row = np.full((1, 1, 1, 8), 0.3)
+    np.testing.assert_allclose(oracle.readout_gate(row, np.full(row.shape, 40.0), eps=0.01),
+                               0.3 / np.sqrt(0.09 + 0.01), rtol=1e-14)
