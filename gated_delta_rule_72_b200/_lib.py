@@ -27,6 +27,7 @@ SIGNATURES = {
                                    _P, _Z, _P]),
     "gdn_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "gdn_step_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "gdn_readout_gate": (_I, [_P, _I, _P, _I, _P, ctypes.c_float, _P, _I, _I, _I, _I, _I, _P]),
     "gdn_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gdn_status_string": (ctypes.c_char_p, [_I]),
     "gdn_version": (ctypes.c_char_p, []),
@@ -120,6 +121,10 @@ def gdn_device_timeouts():
 
 def gdn_launch_count():
     return int(load().gdn_launch_count())
+
+
+def gdn_readout_gate(o, o_dt, z, z_dt, gamma, eps, y, y_dt, B, T, H, dv, stream):
+    return load().gdn_readout_gate(o, o_dt, z, z_dt, gamma, eps, y, y_dt, B, T, H, dv, stream)
 
 
 def gdn_set_kernel_timing(on):

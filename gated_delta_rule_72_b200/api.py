@@ -134,3 +134,30 @@ def step(q, k, v, alpha, beta, state, *, out=None, out_dtype=torch.float32, work
                        B, T, H, dk, dv, dt, odt, _ptr(ws), nbytes, stream)
     _raise("gdn_step", st)
     return o
+
+
+def readout_gate(o, z, gamma=None, eps=1e-6, *, out=None, out_dtype=None):
+    """Readout epilogue: y = o / sqrt(mean(o^2 over d_v) + eps) * gamma * sigmoid(z),
+    per (b, t, h).  o, z: [B,T,H,dv] (fp32 or bf16); gamma: [dv] fp32 or None.
+    y is `out` (may be o or z itself, same dtype) or a new tensor of
+    out_dtype (default: o's dtype)."""
+    _check(o, "o")
+    if o.dtype not in _DT:
+        raise ValueError("o must be float32 or bfloat16")
+    B, T, H, dv = o.shape
+    _check(z, "z", None, (B, T, H, dv))
+    if z.dtype not in _DT:
+        raise ValueError("z must be float32 or bfloat16")
+    if gamma is not None:
+        _check(gamma, "gamma", torch.float32, (dv,))
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=out_dtype or o.dtype, device=o.device)
+    else:
+        _check(out, "out", None, (B, T, H, dv))
+    if out.dtype not in _DT:
+        raise ValueError("out must be float32 or bfloat16")
+    stream = torch.cuda.current_stream(o.device).cuda_stream
+    st = _lib.gdn_readout_gate(_ptr(o), _DT[o.dtype], _ptr(z), _DT[z.dtype], _ptr(gamma), float(eps),
+                               _ptr(out), _DT[out.dtype], B, T, H, dv, stream)
+    _raise("gdn_readout_gate", st)
+    return out

@@ -17,6 +17,7 @@
 #include "tc_chain.cuh"
 #include "tc_fused.cuh"
 #include "tc_prep.cuh"
+#include "readout.cuh"
 #include "token_step.cuh"
 
 // Count of bounded device-side waits that gave up (see gdn_device_timeouts).
@@ -530,6 +531,45 @@ gdn_status run(const Args &a, int bidir) {
     return a.dt == GDN_F32 ? dispatch_out<float>(a, bidir) : dispatch_out<__nv_bfloat16>(a, bidir);
 }
 
+// ---------------------------------------------------------------------------
+// Readout epilogue (readout.cuh)
+// ---------------------------------------------------------------------------
+template <int DV, typename To, typename Tz, typename Ty>
+gdn_status run_readout(const void *o, const void *z, const float *gamma, float eps, void *y, long long rows,
+                       cudaStream_t stream) {
+    const long long per_block = gdn::rd::kThreads / 32;
+    long long blocks = (rows + per_block - 1) / per_block;
+    const long long cap = (long long)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    gdn::LaunchScope ls("readout", stream);
+    gdn::rd::readout_kernel<DV, To, Tz, Ty><<<(int)blocks, gdn::rd::kThreads, 0, stream>>>(
+        static_cast<const To *>(o), static_cast<const Tz *>(z), gamma, eps, static_cast<Ty *>(y), rows);
+    return launch_status();
+}
+
+template <int DV, typename To, typename Tz>
+gdn_status readout_y(gdn_dtype y_dt, const void *o, const void *z, const float *gamma, float eps, void *y,
+                     long long rows, cudaStream_t s) {
+    return y_dt == GDN_F32 ? run_readout<DV, To, Tz, float>(o, z, gamma, eps, y, rows, s)
+                           : run_readout<DV, To, Tz, __nv_bfloat16>(o, z, gamma, eps, y, rows, s);
+}
+
+template <int DV, typename To>
+gdn_status readout_z(gdn_dtype z_dt, gdn_dtype y_dt, const void *o, const void *z, const float *gamma, float eps,
+                     void *y, long long rows, cudaStream_t s) {
+    return z_dt == GDN_F32 ? readout_y<DV, To, float>(y_dt, o, z, gamma, eps, y, rows, s)
+                           : readout_y<DV, To, __nv_bfloat16>(y_dt, o, z, gamma, eps, y, rows, s);
+}
+
+template <int DV>
+gdn_status readout_o(gdn_dtype o_dt, gdn_dtype z_dt, gdn_dtype y_dt, const void *o, const void *z,
+                     const float *gamma, float eps, void *y, long long rows, cudaStream_t s) {
+    return o_dt == GDN_F32 ? readout_z<DV, float>(z_dt, y_dt, o, z, gamma, eps, y, rows, s)
+                           : readout_z<DV, __nv_bfloat16>(z_dt, y_dt, o, z, gamma, eps, y, rows, s);
+}
+
+size_t dtype_bytes(gdn_dtype d) { return d == GDN_F32 ? 4 : 2; }
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -702,4 +742,31 @@ int gdn_read_kernel_timing(char *names, int name_len, double *total_ms, int *lau
     return status == GDN_OK ? n : status;
 }
 
+gdn_status gdn_readout_gate(const void *o, gdn_dtype o_dt, const void *z, gdn_dtype z_dt, const float *gamma,
+                            float eps, void *y, gdn_dtype y_dt, int B, int T, int H, int dv, void *stream) {
+    const gdn_dtype dts[3] = {o_dt, z_dt, y_dt};
+    for (gdn_dtype d : dts)
+        if (d != GDN_F32 && d != GDN_BF16) return GDN_ERR_DTYPE;
+    if (B < 1 || H < 1 || T < 0 || (long long)B * H > 65535LL || T > (1 << 30)) return GDN_ERR_SHAPE;
+    if (dv != 64 && dv != 128) return GDN_ERR_UNSUPPORTED;
+    if (!(eps >= 0.f) || eps > 3.0e38f) return GDN_ERR_SHAPE;   // also rejects NaN
+    if (T == 0) return GDN_OK;
+    if (!o || !z || !y) return GDN_ERR_NULL;
+    if (!aligned(o, 16) || !aligned(z, 16) || !aligned(y, 16) || (gamma && !aligned(gamma, 4)))
+        return GDN_ERR_ALIGN;
+    // y may be o or z itself (same dtype); no other overlap
+    const long long rows = (long long)B * T * H;
+    auto span = [&](const void *p, gdn_dtype d) { return (size_t)rows * dv * dtype_bytes(d); };
+    auto overlap = [](const void *a, size_t na, const void *b, size_t nb) {
+        const char *p = static_cast<const char *>(a), *q = static_cast<const char *>(b);
+        return p < q + nb && q < p + na;
+    };
+    if (overlap(y, span(y, y_dt), o, span(o, o_dt)) && !(y == o && y_dt == o_dt)) return GDN_ERR_SHAPE;
+    if (overlap(y, span(y, y_dt), z, span(z, z_dt)) && !(y == z && y_dt == z_dt)) return GDN_ERR_SHAPE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return dv == 128 ? readout_o<128>(o_dt, z_dt, y_dt, o, z, gamma, eps, y, rows, s)
+                     : readout_o<64>(o_dt, z_dt, y_dt, o, z, gamma, eps, y, rows, s);
+}
+
 }  // extern "C"
+

@@ -197,6 +197,25 @@ GDN_API size_t gdn_workspace_size(int B, int T, int H, int dk, int dv, gdn_dtype
  */
 GDN_API int gdn_set_short_call_tokens(int max_t);
 
+/*
+ * gdn_readout_gate -- readout epilogue of the linear branch, one pass over o:
+ *   y[b,t,h,:] = o[b,t,h,:] / sqrt(mean_j o[b,t,h,j]^2 + eps) * gamma * sigmoid(z[b,t,h,:])
+ * i.e. an RMS norm over the head's dv channels of each token, a per-channel
+ * gain gamma ([dv] fp32; NULL = ones) and the content-dependent sigmoid gate
+ * z.  Source: AI summary of "Video DeltaNet: A Video-Native Hybrid Attention
+ * for Livestream Video Generation", "Key Contributions" 1 (the linear branch
+ * has its own sigmoid gate and an RMS-normalised readout; the axis and the
+ * order, norm then gate, are this library's reading).
+ *   o, z, y: [B, T, H, dv] contiguous, dtypes o_dt, z_dt, y_dt (GDN_F32 or
+ *   GDN_BF16), 16-byte aligned; dv in {64, 128}; eps >= 0 and finite.  y may
+ *   be o or z itself when its dtype matches (in place); any other overlap is
+ *   GDN_ERR_SHAPE.  T = 0 is a no-op.  Asynchronous on `stream`; no
+ *   workspace.  All arithmetic in fp32.
+ */
+GDN_API gdn_status gdn_readout_gate(const void *o, gdn_dtype o_dt, const void *z, gdn_dtype z_dt,
+                                    const float *gamma, float eps, void *y, gdn_dtype y_dt,
+                                    int B, int T, int H, int dv, void *stream);
+
 /* gdn_status_string -- static, NUL-terminated description of a status. */
 GDN_API const char *gdn_status_string(gdn_status s);
 

@@ -178,3 +178,28 @@ def test_bidir_states_rejects_before_launch(lib):
     # each direction in place, or four separate buffers: only the workspace is short
     assert _bidir_states(state_in=A, state_out=A, state_in_bwd=Bb, state_out_bwd=Bb) == -6
     assert _bidir_states(state_in=A, state_in_bwd=Bb, state_out=C, state_out_bwd=D) == -6
+
+
+def _readout(**kw):
+    a = dict(o=FAKE, o_dt=0, z=FAKE, z_dt=0, gamma=None, eps=1e-6, y=FAKE + (1 << 20), y_dt=0, B=1, T=8, H=2,
+             dv=64, stream=None)
+    a.update(kw)
+    return _lib.gdn_readout_gate(*a.values())
+
+
+def test_readout_rejects_before_launch(lib):
+    """gdn_readout_gate argument checks (no CUDA call on these paths)."""
+    assert _readout(o_dt=3) == -3
+    assert _readout(y_dt=-1) == -3
+    assert _readout(dv=96) == -5
+    assert _readout(B=0) == -2
+    assert _readout(eps=-1.0) == -2
+    assert _readout(eps=float("nan")) == -2
+    assert _readout(o=None) == -1
+    assert _readout(z=FAKE + 8) == -4
+    assert _readout(gamma=FAKE + 2) == -4
+    # y over part of o, or over o with another dtype
+    assert _readout(y=FAKE + 256) == -2
+    assert _readout(y=FAKE, y_dt=1) == -2
+    # T = 0: nothing to do, no pointer needed
+    assert _readout(T=0, o=None, z=None, y=None) == 0

@@ -356,3 +356,48 @@ def test_rollout_replays_in_a_cuda_graph():
     o_ref, s_ref = oracle_heads(inp)
     assert rel_err(o_g, o_ref) <= TOL[torch.bfloat16]
     assert rel_err(s_g, s_ref) <= TOL[torch.bfloat16]
+
+
+
+DTS = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@pytest.mark.parametrize("dv", [64, 128])
+@pytest.mark.parametrize("o_dt,z_dt,y_dt", [("f32", "f32", "f32"), ("f32", "bf16", "bf16"),
+                                            ("bf16", "f32", "f32"), ("bf16", "bf16", "bf16")])
+@pytest.mark.parametrize("eps,with_gamma", [(1e-6, False), (0.1, True)])
+def test_readout_gate(dv, o_dt, z_dt, y_dt, eps, with_gamma):
+    """Readout epilogue against the oracle, ragged row count (B*T*H = 222)."""
+    from oracle import readout_gate as ref_readout
+    B, T, H = 2, 37, 3
+    g = torch.Generator("cpu").manual_seed(dv + len(o_dt + z_dt + y_dt))
+    o = (torch.randn(B, T, H, dv, generator=g) * torch.rand(B, T, H, 1, generator=g) * 3).to(DTS[o_dt])
+    z = (2 * torch.randn(B, T, H, dv, generator=g)).to(DTS[z_dt])
+    gamma = (0.5 + torch.rand(dv, generator=g)) if with_gamma else None
+    y = gdn.readout_gate(o.cuda(), z.cuda(), None if gamma is None else gamma.cuda(), eps,
+                         out_dtype=DTS[y_dt])
+    torch.cuda.synchronize()
+    want = ref_readout(o, z, gamma, eps)
+    if y_dt == "f32":
+        assert rel_err(y, want) <= 1e-4
+    else:
+        assert rel_err_bf16_out(y, want) <= 1e-4
+
+
+def test_readout_in_place_after_a_scan():
+    """The linear branch end to end: causal scan, then the readout written
+    over the scan's fp32 output in place; against oracle scan + readout."""
+    from oracle import readout_gate as ref_readout
+    B, T, H, dk, dv = 1, 300, 4, 128, 128
+    inp = inputs.generate(B, T, H, dk, dv, "bf16", seed=123)
+    d = to_dev(inp)
+    o, _ = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+    g = torch.Generator("cpu").manual_seed(5)
+    z = torch.randn(B, T, H, dv, generator=g)
+    gamma = 0.5 + torch.rand(dv, generator=g)
+    y = gdn.readout_gate(o, z.cuda(), gamma.cuda(), 1e-6, out=o)
+    torch.cuda.synchronize()
+    assert y.data_ptr() == o.data_ptr()
+    o_ref, _ = oracle_heads(inp)
+    want = ref_readout(o_ref, z, gamma, 1e-6)
+    assert rel_err(y, want) <= TOL[torch.bfloat16]
