@@ -119,3 +119,64 @@ def readout_gate(o, z, gamma=None, eps=1e-6):
         for j in range(dv):
             flat_y[r, j] = row[j] * inv * g[j] / (1.0 + np.exp(-flat_z[r, j]))
     return y
+
+
+def vda_scan(q, k, v, alpha_f, beta, U, mode="causal", state_in=None, state_in_bwd=None):
+    """Frame-wise delta operator (VDA), in float64.  The sequence is split
+    into frames of U consecutive tokens (T = F * U).  For frame f with keys
+    K_f (U x dk), values V_f (U x dv), per-token write strengths beta and a
+    per-frame decay alpha_f:
+
+        A_f = K_f^T diag(beta) K_f,   B_f = K_f^T diag(beta) V_f
+        S_f = (I + A_f)^{-1} (alpha_f S_{f-1} + B_f)
+
+    the minimiser of ||S - alpha_f S_{f-1}||^2 + sum_u beta_u ||S^T k_u - v_u||^2:
+    the state that stays close to the decayed memory while fitting every
+    key-value pair of the frame at once.  Causal readout: o_u = S_f^T q_u for
+    the tokens u of frame f.  Reverse (strict): R_f = (I + A_f)^{-1}
+    (alpha_f R_{f+1} + B_f) from R_{F+1} = state_in_bwd, read as
+    o_u = R_{f+1}^T q_u (the frames after f only); bidir adds the two.
+
+    Source: AI summary of "Video DeltaNet: A Video-Native Hybrid Attention for
+    Livestream Video Generation", "Key Contributions" 2 (the closed form
+    S_t = (S_bar_t + B_t)(I + A_t)^{-1}, written there for a state that maps
+    keys to values, i.e. the transpose of the layout here) and "Methodology in
+    Plain English" (the least-squares objective in words).  The pages leave
+    S_bar, A and B undefined; the reading here (S_bar = decayed previous state,
+    A and B the frame's beta-weighted key Gram and key-value products) is the
+    one that objective gives.  np.linalg.solve is the library step.
+
+    q, k: [B, T, H, dk]; v: [B, T, H, dv]; alpha_f: [B, F, H]; beta: [B, T, H].
+    Returns (o [B, T, H, dv], S_F or None, R_1 or None), float64."""
+    q, k, v, alpha_f, beta = (_f64(x) for x in (q, k, v, alpha_f, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert U >= 1 and T % U == 0
+    F = T // U
+    assert alpha_f.shape == (B, F, H) and beta.shape == (B, T, H)
+    s0, r0 = _f64(state_in), _f64(state_in_bwd)
+    o = np.zeros((B, T, H, dv))
+    sf = np.zeros((B, H, dk, dv)) if mode in ("causal", "bidir") else None
+    sb = np.zeros((B, H, dk, dv)) if mode in ("reverse", "bidir") else None
+    eye = np.eye(dk)
+    for b in range(B):
+        for h in range(H):
+            def frame(f):
+                t = slice(f * U, (f + 1) * U)
+                K, V, be = k[b, t, h], v[b, t, h], beta[b, t, h]
+                return t, K.T @ (be[:, None] * K), K.T @ (be[:, None] * V)
+            if mode in ("causal", "bidir"):
+                S = np.zeros((dk, dv)) if s0 is None else s0[b, h].copy()
+                for f in range(F):
+                    t, A, Bm = frame(f)
+                    S = np.linalg.solve(eye + A, alpha_f[b, f, h] * S + Bm)
+                    o[b, t, h] += q[b, t, h] @ S
+                sf[b, h] = S
+            if mode in ("reverse", "bidir"):
+                R = np.zeros((dk, dv)) if r0 is None else r0[b, h].copy()
+                for f in range(F - 1, -1, -1):
+                    t, A, Bm = frame(f)
+                    o[b, t, h] += q[b, t, h] @ R
+                    R = np.linalg.solve(eye + A, alpha_f[b, f, h] * R + Bm)
+                sb[b, h] = R
+    return o, sf, sb

@@ -350,3 +350,111 @@ def test_readout_normalises_and_gates():
     row = np.full((1, 1, 1, 8), 0.3)
     np.testing.assert_allclose(oracle.readout_gate(row, np.full(row.shape, 40.0), eps=0.01),
                                0.3 / np.sqrt(0.09 + 0.01), rtol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# frame-wise delta operator (VDA)
+# --------------------------------------------------------------------------
+def _vda_inputs(rng, B, F, U, H, dk, dv, unit=True):
+    q = rng.normal(size=(B, F * U, H, dk))
+    k = rng.normal(size=(B, F * U, H, dk))
+    if unit:
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.normal(size=(B, F * U, H, dv))
+    a = rng.uniform(0.5, 1.0, size=(B, F, H))
+    b = rng.uniform(0.0, 1.0, size=(B, F * U, H))
+    return q, k, v, a, b
+
+
+@pytest.mark.parametrize("unit", [True, False])
+def test_vda_one_token_frames_are_the_delta_rule(unit):
+    """U = 1: (I + b k k^T)^{-1} = I - c k k^T with c = b / (1 + b |k|^2), so a
+    frame step is the gated delta rule with erase = write = c (Sherman-Morrison);
+    checked against the token recurrence of the C oracle, causal and bidir."""
+    rng = np.random.default_rng(31)
+    q, k, v, a, b = _vda_inputs(rng, 2, 11, 1, 2, 5, 3, unit=unit)
+    c = b / (1.0 + b * np.sum(k * k, axis=-1))
+    S0 = rng.normal(size=(2, 2, 5, 3))
+    R0 = rng.normal(size=(2, 2, 5, 3))
+    for mode in ("causal", "bidir"):
+        o, sf, sb = oracle.vda_scan(q, k, v, a, b, 1, mode=mode, state_in=S0, state_in_bwd=R0)
+        o2, sf2, sb2 = oracle.scan(q, k, v, a, b, mode=mode, state_in=S0, state_in_bwd=R0, erase=c, write=c)
+        np.testing.assert_allclose(o, o2, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(sf, sf2, rtol=1e-10, atol=1e-12)
+        if mode == "bidir":
+            np.testing.assert_allclose(sb, sb2, rtol=1e-10, atol=1e-12)
+
+
+def test_vda_orthonormal_frame_is_a_token_scan():
+    """A frame whose U keys are orthonormal: the key directions decouple, so
+    the frame step equals the token-level delta rule over the frame's tokens
+    with erase = write = b_u / (1 + b_u), the frame's decay applied at its
+    first token only (and 1 at the others); the readout is that of the frame's
+    final state."""
+    rng = np.random.default_rng(32)
+    B, F, U, H, dk, dv = 1, 4, 3, 1, 6, 2
+    q, k, v, a, b = _vda_inputs(rng, B, F, U, H, dk, dv)
+    for f in range(F):   # orthonormal keys within each frame
+        Qm, _ = np.linalg.qr(rng.normal(size=(dk, U)))
+        k[0, f * U:(f + 1) * U, 0] = Qm.T
+    c = b / (1.0 + b)
+    a_tok = np.ones((B, F * U, H))
+    a_tok[:, ::U] = a
+    S0 = rng.normal(size=(B, H, dk, dv))
+    o, sf, _ = oracle.vda_scan(q, k, v, a, b, U, state_in=S0)
+    _, S_tok, _ = oracle.scan(q, k, v, a_tok, b, state_in=S0, erase=c, write=c)
+    np.testing.assert_allclose(sf, S_tok, rtol=1e-10, atol=1e-12)
+    # readout per frame: every token of frame f reads the state after the frame
+    S = S0[0, 0]
+    for f in range(F):
+        t = slice(f * U, (f + 1) * U)
+        _, S_f, _ = oracle.scan(q[:, :(f + 1) * U], k[:, :(f + 1) * U], v[:, :(f + 1) * U],
+                                a_tok[:, :(f + 1) * U], b[:, :(f + 1) * U], state_in=S0,
+                                erase=c[:, :(f + 1) * U], write=c[:, :(f + 1) * U])
+        np.testing.assert_allclose(o[0, t, 0], q[0, t, 0] @ S_f[0, 0], rtol=1e-10, atol=1e-12)
+
+
+def test_vda_inherited_state_is_not_amplified():
+    """With zero values (B_f = 0) a frame step maps S to alpha (I + A)^{-1} S,
+    whose spectral norm is at most alpha: ||S_f||_2 <= alpha_f ||S_{f-1}||_2,
+    whatever the keys (non-unit keys with large write strengths included)."""
+    rng = np.random.default_rng(33)
+    B, F, U, H, dk, dv = 1, 6, 40, 1, 8, 8
+    q, k, v, a, b = _vda_inputs(rng, B, F, U, H, dk, dv, unit=False)
+    k *= 3.0
+    v[:] = 0.0
+    S = rng.normal(size=(B, H, dk, dv))
+    for f in range(F):
+        sl = slice(f * U, (f + 1) * U)
+        _, S_next, _ = oracle.vda_scan(q[:, sl], k[:, sl], v[:, sl], a[:, f:f + 1], b[:, sl], U, state_in=S)
+        assert np.linalg.norm(S_next[0, 0], 2) <= a[0, f, 0] * np.linalg.norm(S[0, 0], 2) * (1 + 1e-12)
+        S = S_next
+
+
+def test_vda_reverse_is_causal_on_reversed_frames():
+    """The reverse readout of frame f is the causal state of the frames after
+    f taken in reverse order (from R_{F+1}); R_1 is that of all frames."""
+    rng = np.random.default_rng(34)
+    B, F, U, H, dk, dv = 1, 5, 4, 2, 5, 3
+    q, k, v, a, b = _vda_inputs(rng, B, F, U, H, dk, dv)
+    R0 = rng.normal(size=(B, H, dk, dv))
+    o, _, R1 = oracle.vda_scan(q, k, v, a, b, U, mode="reverse", state_in_bwd=R0)
+
+    def rev_frames(x, per_frame=False):   # reverse the frame order, keep token order inside a frame
+        if per_frame:
+            return x[:, ::-1]
+        n = x.shape[1] // U
+        return np.concatenate([x[:, f * U:(f + 1) * U] for f in range(n - 1, -1, -1)], axis=1)
+
+    for f in range(F):
+        t = slice(f * U, (f + 1) * U)
+        if f + 1 < F:
+            suf = slice((f + 1) * U, F * U)
+            _, S, _ = oracle.vda_scan(rev_frames(q[:, suf]), rev_frames(k[:, suf]), rev_frames(v[:, suf]),
+                                      rev_frames(a[:, f + 1:], True), rev_frames(b[:, suf]), U, state_in=R0)
+        else:
+            S = R0
+        np.testing.assert_allclose(o[0, t], np.einsum("thi,hij->thj", q[0, t], S[0]), rtol=1e-10, atol=1e-12)
+    _, S_all, _ = oracle.vda_scan(rev_frames(q), rev_frames(k), rev_frames(v), rev_frames(a, True),
+                                  rev_frames(b), U, state_in=R0)
+    np.testing.assert_allclose(R1, S_all, rtol=1e-10, atol=1e-12)
