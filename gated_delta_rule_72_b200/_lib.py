@@ -27,6 +27,9 @@ SIGNATURES = {
                                    _P, _Z, _P]),
     "gdn_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "gdn_step_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "gdn_vda_scan": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P,
+                          _Z, _P]),
+    "gdn_vda_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I]),
     "gdn_readout_gate": (_I, [_P, _I, _P, _I, _P, ctypes.c_float, _P, _I, _I, _I, _I, _I, _P]),
     "gdn_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gdn_status_string": (ctypes.c_char_p, [_I]),
@@ -121,6 +124,16 @@ def gdn_device_timeouts():
 
 def gdn_launch_count():
     return int(load().gdn_launch_count())
+
+
+def gdn_vda_scan(q, k, v, alpha_frame, beta, state_in, state_in_bwd, state_out, state_out_bwd, o, B, F, U, H,
+                 dk, dv, bidir, dt, o_dt, workspace, ws_bytes, stream):
+    return load().gdn_vda_scan(q, k, v, alpha_frame, beta, state_in, state_in_bwd, state_out, state_out_bwd, o,
+                               B, F, U, H, dk, dv, bidir, dt, o_dt, workspace, ws_bytes, stream)
+
+
+def gdn_vda_workspace_size(B, F, U, H, dk, dv, bidir):
+    return int(load().gdn_vda_workspace_size(B, F, U, H, dk, dv, int(bool(bidir))))
 
 
 def gdn_readout_gate(o, o_dt, z, z_dt, gamma, eps, y, y_dt, B, T, H, dv, stream):

@@ -161,3 +161,41 @@ def readout_gate(o, z, gamma=None, eps=1e-6, *, out=None, out_dtype=None):
                                _ptr(out), _DT[out.dtype], B, T, H, dv, stream)
     _raise("gdn_readout_gate", st)
     return out
+
+
+def vda_scan(q, k, v, alpha_frame, beta, U, *, bidir=False, state=None, state_bwd=None, return_states=False,
+             out=None, out_dtype=torch.float32, workspace=None):
+    """Frame-wise delta operator over frames of U tokens (T = F * U):
+    S_f = (I + K^T diag(beta) K)^{-1} (alpha_f S_{f-1} + K^T diag(beta) V), read by
+    every token of frame f (bidir: plus the reverse scan, read strictly).
+    alpha_frame: [B, F, H] fp32; beta: [B, T, H] fp32.  Returns o, or with
+    return_states (o, S_F, R_1) (R_1 None unless bidir)."""
+    if q.dtype not in _DT:
+        raise ValueError("q must be float32 or bfloat16")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if U < 1 or T % U != 0:
+        raise ValueError("T (%d) must be a multiple of the frame length U (%d)" % (T, U))
+    F = T // U
+    _check(q, "q")
+    _check(k, "k", q.dtype, (B, T, H, dk))
+    _check(v, "v", q.dtype, (B, T, H, dv))
+    _check(alpha_frame, "alpha_frame", torch.float32, (B, F, H))
+    _check(beta, "beta", torch.float32, (B, T, H))
+    for t, name in ((state, "state"), (state_bwd, "state_bwd")):
+        if t is not None:
+            _check(t, name, torch.float32, (B, H, dk, dv))
+    o, odt = _out(B, T, H, dv, q.device, out, out_dtype)
+    s_out = s_out_b = None
+    if return_states:
+        s_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+        if bidir:
+            s_out_b = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    ws, nbytes = _workspace(int(_lib.gdn_vda_workspace_size(B, F, U, H, dk, dv, int(bool(bidir)))), q.device,
+                            workspace)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    st = _lib.gdn_vda_scan(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha_frame), _ptr(beta), _ptr(state),
+                           _ptr(state_bwd), _ptr(s_out), _ptr(s_out_b), _ptr(o), B, F, U, H, dk, dv,
+                           int(bool(bidir)), _DT[q.dtype], odt, _ptr(ws), nbytes, stream)
+    _raise("gdn_vda_scan", st)
+    return (o, s_out, s_out_b) if return_states else o

@@ -19,6 +19,7 @@
 #include "tc_prep.cuh"
 #include "readout.cuh"
 #include "token_step.cuh"
+#include "vda.cuh"
 
 // Count of bounded device-side waits that gave up (see gdn_device_timeouts).
 static __device__ unsigned int g_wait_timeouts;
@@ -570,6 +571,76 @@ gdn_status readout_o(gdn_dtype o_dt, gdn_dtype z_dt, gdn_dtype y_dt, const void 
 
 size_t dtype_bytes(gdn_dtype d) { return d == GDN_F32 ? 4 : 2; }
 
+// ---------------------------------------------------------------------------
+// Frame-wise delta operator (vda.cuh)
+// ---------------------------------------------------------------------------
+struct VdaArgs {
+    const void *q, *k, *v;
+    const float *alpha_f, *beta;
+    const float *s_in, *s_in_bwd;
+    float *s_out, *s_out_bwd;
+    void *o;
+    int B, F, U, H, dk, dv, bidir;
+    gdn_dtype dt, o_dt;
+    void *ws;
+    size_t ws_bytes;
+    cudaStream_t stream;
+};
+
+// workspace: A [F][B*H][dk][dk], B [F][B*H][dk][dv], states [ndir][F][B*H][dk][dv]
+size_t vda_workspace(int B, int F, int H, int dk, int dv, int bidir) {
+    const size_t fh = (size_t)F * B * H;
+    return round_up(fh * dk * dk * 4, 256) + round_up(fh * dk * dv * 4, 256) +
+           round_up((bidir ? 2 : 1) * fh * dk * dv * 4, 256);
+}
+
+template <int DK, int DV, typename Tin, typename Tout>
+gdn_status run_vda(const VdaArgs &a) {
+    using namespace gdn::vda;
+    const int nbh = a.B * a.H, ndir = a.bidir ? 2 : 1;
+    const size_t fh = (size_t)a.F * nbh;
+    float *A = static_cast<float *>(a.ws);
+    float *Bm = reinterpret_cast<float *>(static_cast<char *>(a.ws) + round_up(fh * DK * DK * 4, 256));
+    float *st = reinterpret_cast<float *>(reinterpret_cast<char *>(Bm) + round_up(fh * DK * DV * 4, 256));
+    {
+        auto kern = vda_gram_kernel<DK, DV, Tin>;
+        constexpr int smem = GramSmem<DK, DV>::kBytes;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        gdn::LaunchScope ls("vda_gram", a.stream);
+        kern<<<dim3(a.F, nbh), kThreads, smem, a.stream>>>(static_cast<const Tin *>(a.k), static_cast<const Tin *>(a.v),
+                                                          a.beta, A, Bm, a.F, a.U, a.H);
+        if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
+    }
+    {
+        auto kern = vda_chain_kernel<DK, DV>;
+        constexpr int smem = ChainSmem<DK, DV>::kBytes;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        gdn::LaunchScope ls("vda_chain", a.stream);
+        kern<<<dim3(nbh, ndir), kChainThreads, smem, a.stream>>>(A, Bm, a.alpha_f, a.s_in, a.s_in_bwd, a.s_out,
+                                                                a.s_out_bwd, st, a.F, a.H);
+        if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
+    }
+    auto kern = vda_readout_kernel<DK, DV, Tin, Tout>;
+    const int smem = ndir == 2 ? ReadSmem<DK, DV>::kBytes2 : ReadSmem<DK, DV>::kBytes1;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, ReadSmem<DK, DV>::kBytes2) !=
+        cudaSuccess)
+        return GDN_ERR_CUDA;
+    gdn::LaunchScope ls("vda_readout", a.stream);
+    kern<<<dim3(a.F * ((a.U + 63) / 64), nbh), kThreads, smem, a.stream>>>(
+        static_cast<const Tin *>(a.q), st, static_cast<Tout *>(a.o), a.F, a.U, a.H, ndir);
+    return launch_status();
+}
+
+template <typename Tin, typename Tout>
+gdn_status vda_dims(const VdaArgs &a) {
+    if (a.dk == 128 && a.dv == 128) return run_vda<128, 128, Tin, Tout>(a);
+    if (a.dk == 128 && a.dv == 64) return run_vda<128, 64, Tin, Tout>(a);
+    if (a.dk == 64 && a.dv == 128) return run_vda<64, 128, Tin, Tout>(a);
+    return run_vda<64, 64, Tin, Tout>(a);
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -740,6 +811,32 @@ int gdn_read_kernel_timing(char *names, int name_len, double *total_ms, int *lau
     }
     st.events.clear();
     return status == GDN_OK ? n : status;
+}
+
+gdn_status gdn_vda_scan(const void *q, const void *k, const void *v, const float *alpha_frame, const float *beta,
+                        const float *state_in, const float *state_in_bwd, float *state_out, float *state_out_bwd,
+                        void *o, int B, int F, int U, int H, int dk, int dv, int bidir, gdn_dtype dt,
+                        gdn_dtype o_dt, void *workspace, size_t ws_bytes, void *stream) {
+    // the argument rules of the token scans, with T = F * U
+    if (U < 1 || F < 0 || (long long)F * U > (1 << 30)) return GDN_ERR_SHAPE;
+    Args c{q, k, v, alpha_frame, beta, state_in, state_out, o, B, F * U, H, dk, dv, dt, o_dt,
+           workspace, ws_bytes, static_cast<cudaStream_t>(stream), bidir ? state_in_bwd : nullptr,
+           bidir ? state_out_bwd : nullptr};
+    gdn_status s = check_common(c, F > 0);
+    if (s != GDN_OK) return s;
+    if ((long long)F * B * H > 65535LL * 64) return GDN_ERR_SHAPE;
+    if (F == 0) return empty_scan(c, bidir ? 1 : 0);
+    s = check_ws(c, vda_workspace(B, F, H, dk, dv, bidir ? 1 : 0));
+    if (s != GDN_OK) return s;
+    const VdaArgs a{q, k, v, alpha_frame, beta, state_in, c.state_in_bwd, state_out, c.state_out_bwd, o,
+                    B, F, U, H, dk, dv, bidir ? 1 : 0, dt, o_dt, workspace, ws_bytes, c.stream};
+    if (dt == GDN_F32) return o_dt == GDN_F32 ? vda_dims<float, float>(a) : vda_dims<float, __nv_bfloat16>(a);
+    return o_dt == GDN_F32 ? vda_dims<__nv_bfloat16, float>(a) : vda_dims<__nv_bfloat16, __nv_bfloat16>(a);
+}
+
+size_t gdn_vda_workspace_size(int B, int F, int U, int H, int dk, int dv, int bidir) {
+    if (B < 1 || H < 1 || F < 0 || U < 1 || !((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return 0;
+    return F == 0 ? 0 : vda_workspace(B, F, H, dk, dv, bidir ? 1 : 0);
 }
 
 gdn_status gdn_readout_gate(const void *o, gdn_dtype o_dt, const void *z, gdn_dtype z_dt, const float *gamma,

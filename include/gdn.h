@@ -198,6 +198,39 @@ GDN_API size_t gdn_workspace_size(int B, int T, int H, int dk, int dv, gdn_dtype
 GDN_API int gdn_set_short_call_tokens(int max_t);
 
 /*
+ * gdn_vda_scan -- the frame-wise delta operator: the sequence is F frames of
+ * U consecutive tokens (T = F * U) and the state is written once per frame,
+ * by all of the frame's tokens at once:
+ *   A_f = K_f^T diag(beta) K_f,   B_f = K_f^T diag(beta) V_f
+ *   S_f = (I + A_f)^{-1} (alpha_f S_{f-1} + B_f),   o_u = S_f^T q_u  (u in frame f)
+ * S_f is the state closest to the decayed memory alpha_f S_{f-1} that fits
+ * every key-value pair of the frame in the least-squares sense (weights
+ * beta).  bidir != 0 adds the reverse scan R_f = (I + A_f)^{-1} (alpha_f
+ * R_{f+1} + B_f) read strictly: o_u += R_{f+1}^T q_u (the frames after f).
+ * Source: AI summary of "Video DeltaNet: A Video-Native Hybrid Attention for
+ * Livestream Video Generation", "Key Contributions" 2 (the closed form, for
+ * a state mapping keys to values, i.e. the transpose of this layout) and
+ * "Methodology in Plain English" (the objective in words); A_f, B_f and the
+ * decayed previous state are this library's reading of that objective.
+ *   q, k [B, T, H, dk]; v, o [B, T, H, dv] (dtypes dt, o_dt); alpha_frame
+ *   [B, F, H] fp32 in (0, 1]; beta [B, T, H] fp32 >= 0; states [B, H, dk, dv]
+ *   fp32: state_in / state_out the causal S_0 / S_F, state_in_bwd /
+ *   state_out_bwd the reverse R_{F+1} / R_1 (used only when bidir; NULL: zero /
+ *   not written), with the overlap rules of gdn_scan_bidir_states.
+ *   Workspace: gdn_vda_workspace_size bytes, 256-byte aligned.  F = 0 passes
+ *   the states through.  All arithmetic in fp32 (CUDA cores): a Cholesky
+ *   factorisation of I + A_f per frame and head.
+ */
+GDN_API gdn_status gdn_vda_scan(const void *q, const void *k, const void *v, const float *alpha_frame,
+                                const float *beta, const float *state_in, const float *state_in_bwd,
+                                float *state_out, float *state_out_bwd, void *o, int B, int F, int U,
+                                int H, int dk, int dv, int bidir, gdn_dtype dt, gdn_dtype o_dt,
+                                void *workspace, size_t ws_bytes, void *stream);
+/* gdn_vda_workspace_size -- bytes of workspace gdn_vda_scan needs (0 for
+ * arguments it would reject, or F = 0). */
+GDN_API size_t gdn_vda_workspace_size(int B, int F, int U, int H, int dk, int dv, int bidir);
+
+/*
  * gdn_readout_gate -- readout epilogue of the linear branch, one pass over o:
  *   y[b,t,h,:] = o[b,t,h,:] / sqrt(mean_j o[b,t,h,j]^2 + eps) * gamma * sigmoid(z[b,t,h,:])
  * i.e. an RMS norm over the head's dv channels of each token, a per-channel

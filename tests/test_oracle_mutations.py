@@ -58,6 +58,9 @@ def _pin_functions():
                 out.append((name + "[" + ex["name"] + "]", lambda ex=ex: pins.test_worked_examples(ex)))
         elif name == "test_split_calls_equal_one_call":
             out.append((name, lambda: pins.test_split_calls_equal_one_call(17)))
+        elif name == "test_vda_one_token_frames_are_the_delta_rule":
+            for unit in (True, False):
+                out.append((name + "[%s]" % unit, lambda unit=unit: pins.test_vda_one_token_frames_are_the_delta_rule(unit)))
         else:
             out.append((name, fn))
     return out
