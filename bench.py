@@ -78,10 +78,27 @@ def state_bytes_per_call(w):
 
 def flops_per_token_head(w, C=64):
     dk, dv = w.dk, w.dv
+    if w.mode == "vda":
+        return sum(vda_kernel_flops(w).values())
     causal = C * (6 * dk + 4 * dv) + 6 * dk * dv + C * C / 3.0
     if w.mode == "bidir":
         return causal + C * (2 * dk + 4 * dv) + 6 * dk * dv + C * C / 3.0
     return causal
+
+
+def vda_kernel_flops(w):
+    """FLOPs per token-head of the frame-wise operator's kernels (bidirectional):
+    the frame's key Gram and key-value products once, per direction a Cholesky
+    of I + A (dk^3/3), two triangular solves (2 dk^2 dv) and the right-hand
+    side (2 dk dv) per frame, and the readout (2 dk dv per token)."""
+    dk, dv, U = w.dk, w.dv, w.frame
+    return {"vda_gram": 2.0 * dk * (dk + dv),
+            "vda_chain": 2 * (dk ** 3 / 3.0 + 2.0 * dk * dk * dv + 2.0 * dk * dv) / U,
+            "vda_readout": 2 * 2.0 * dk * dv}
+
+
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA/clk x 2 FLOP x 1.965 GHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def algorithmic_bytes_per_step(w):
@@ -191,7 +208,11 @@ class GPUStep:
         self.o = torch.empty(w.B, w.total_T, w.H, w.dv, dtype=torch.float32, device=device)
         self.state = torch.zeros(w.B, w.H, w.dk, w.dv, dtype=torch.float32, device=device)
         td = self.d["q"].dtype
-        if w.mode == "rollout":
+        if w.mode == "vda":
+            from gated_delta_rule_72_b200 import inputs as I
+            self.d["alpha_frame"] = I.frame_alpha(self.d["alpha"], w.frame)
+            nb = gdn.gdn_vda_workspace_size(w.B, w.T // w.frame, w.frame, w.H, w.dk, w.dv, 1)
+        elif w.mode == "rollout":
             nb = gdn.workspace_size(w.B, w.T, w.H, w.dk, w.dv, td)
             self.slices = []
             for i in range(w.calls):
@@ -213,6 +234,9 @@ class GPUStep:
         elif w.mode == "bidir":
             gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"], out=self.o,
                            workspace=self.ws)
+        elif w.mode == "vda":
+            gdn.vda_scan(d["q"], d["k"], d["v"], d["alpha_frame"], d["beta"], w.frame, bidir=True, out=self.o,
+                         workspace=self.ws)
         else:
             self.state.zero_()
             for part, o in self.slices:
@@ -235,6 +259,10 @@ class GPUStep:
         elif w.mode == "bidir":
             gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"], out=self.o,
                            workspace=self.ws)
+        elif w.mode == "vda":
+            from gated_delta_rule_72_b200 import inputs as I
+            gdn.vda_scan(d["q"], d["k"], d["v"], I.frame_alpha(d["alpha"], w.frame), d["beta"], w.frame,
+                         bidir=True, out=self.o, workspace=self.ws)
         else:
             self.state.zero_()
             for i in range(w.calls):
@@ -296,24 +324,38 @@ def whole_job_value(n_gpus, units_per_gpu, ms_max):
 # ---------------------------------------------------------------------------
 # the FP64 oracle on the host cores (cpu_baseline and --impl reference)
 # ---------------------------------------------------------------------------
-def oracle_sample(w, target_s):
-    """Time the oracle on the first T_s tokens of every head, T_s sized so the
-    run takes about target_s seconds.  Returns (Mtok/s, threads, description)."""
+def oracle_run(w, x, threads):
+    """One oracle pass over the inputs x of workload w (a sample of it)."""
     import oracle
     from gated_delta_rule_72_b200 import inputs
+    if w.mode == "vda":
+        oracle.vda_scan(x["q"], x["k"], x["v"], inputs.frame_alpha(x["alpha"], w.frame), x["beta"], w.frame,
+                        mode="bidir")
+    else:
+        oracle.scan(x["q"], x["k"], x["v"], x["alpha"], x["beta"],
+                    mode="bidir" if w.mode == "bidir" else "causal", threads=threads)
+
+
+def oracle_sample(w, target_s):
+    """Time the oracle on the first T_s tokens of every head (whole frames for
+    the frame-wise operator), T_s sized so the run takes about target_s
+    seconds.  Returns (Mtok/s, threads, description, T_s)."""
+    from gated_delta_rule_72_b200 import inputs
     threads = max(1, min(os.cpu_count() or 1, w.B * w.H))
-    mode = "bidir" if w.mode == "bidir" else "causal"
+    mode = {"bidir": "bidir", "vda": "frame-wise, bidir"}.get(w.mode, "causal")
     full_T = w.total_T
+    step = w.frame if w.mode == "vda" else 1
 
     def run(Ts):
         x = inputs.generate(w.B, Ts, w.H, w.dk, w.dv, w.dtype, w.seed, w.gates)
         t0 = time.perf_counter()
-        oracle.scan(x["q"], x["k"], x["v"], x["alpha"], x["beta"], mode=mode, threads=threads)
+        oracle_run(w, x, threads)
         return time.perf_counter() - t0
 
-    Tc = min(full_T, 128)
+    Tc = min(full_T, max(128, step))
     tc = run(Tc)
     Ts = int(min(full_T, max(Tc, Tc * target_s / max(tc, 1e-6))))
+    Ts = max(step, Ts // step * step)
     ts = run(Ts)
     units = w.B * w.H * Ts
     desc = "%s: all %d heads x first %d of %d tokens (%s), float64, %d threads" % (
@@ -327,7 +369,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="stream480",
-                    choices=["stream480", "bidir720", "rollout", "skewed", "tiny"])
+                    choices=["stream480", "bidir720", "rollout", "skewed", "tiny", "vda480"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target length of the oracle CPU-baseline sample")
@@ -348,7 +390,8 @@ def main():
     config = {"workload": "%s (%s B=%d H=%d T=%d%s d_k=%d d_v=%d, %s in, fp32 out/state, %s gates)"
               % (w.name, w.mode, w.B, w.H, w.T, (" x %d calls" % w.calls) if w.calls > 1 else "",
                  w.dk, w.dv, w.dtype, w.gates),
-              "B": w.B, "H": w.H, "T": w.total_T, "d_k": w.dk, "d_v": w.dv, "chunk": 64,
+              "B": w.B, "H": w.H, "T": w.total_T, "d_k": w.dk, "d_v": w.dv,
+              **({"frame": w.frame} if w.mode == "vda" else {"chunk": 64}),
               "parallelism": "replicas%d (independent (b,h) problems per GPU)" % args.gpus}
 
     if args.impl == "reference":
@@ -360,13 +403,12 @@ def main():
         # W warm-up + K timed steps, each the same bounded sample
         from gated_delta_rule_72_b200 import inputs as I
         x = I.generate(w.B, Ts, w.H, w.dk, w.dv, w.dtype, w.seed, w.gates)
-        mode = "bidir" if w.mode == "bidir" else "causal"
         for _ in range(args.warmup):
-            oracle.scan(x["q"], x["k"], x["v"], x["alpha"], x["beta"], mode=mode, threads=threads)
+            oracle_run(w, x, threads)
         times = []
         for _ in range(args.steps):
             t0 = time.perf_counter()
-            oracle.scan(x["q"], x["k"], x["v"], x["alpha"], x["beta"], mode=mode, threads=threads)
+            oracle_run(w, x, threads)
             times.append(time.perf_counter() - t0)
         step_s = sum(times) / len(times)
         value = w.B * w.H * Ts / step_s / 1e6
@@ -436,7 +478,14 @@ def main():
         launches_per_step = n / args.steps
         units_per_launch = units / launches_per_step
         bound = "tensor" if w.mode == "bidir" and "chain" not in name else "hbm"
-        if bound == "hbm":
+        if w.mode == "vda":
+            bound = "alu"     # fp32 on the CUDA cores
+        if bound == "alu":
+            alg = vda_kernel_flops(w).get(name, 0.0) * units_per_launch
+            achieved = alg / (per_launch_ms * 1e-3) / 1e12
+            peak = FP32_ALU_TFLOPS
+            unit = "TFLOP/s"
+        elif bound == "hbm":
             alg = kernel_algorithmic_bytes(name, w) * units_per_launch
             achieved = alg / (per_launch_ms * 1e-3) / 1e9
             peak = peaks["hbm_gbs"]
@@ -451,8 +500,9 @@ def main():
         traffic = tph * units_per_launch if tph is not None else None
         roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": traffic, "kernel": name,
-                "peak_source": "%s (%s)" % (peak_src, "MEASURED_PEAKS.json" if peak_src == "measured"
-                                            else "pool fallback"),
+                "peak_source": ("derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1.965 GHz" if bound == "alu" else
+                                "%s (%s)" % (peak_src, "MEASURED_PEAKS.json" if peak_src == "measured"
+                                             else "pool fallback")),
                 "kernel_ms_per_launch": per_launch_ms,
                 "kernel_share": tot_ms / total_ms if total_ms else None,
                 "kernels": {k: {"ms_per_step": t / args.steps, "launches_per_step": c / args.steps}

@@ -623,9 +623,8 @@ gdn_status run_vda(const VdaArgs &a) {
         if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
     }
     auto kern = vda_readout_kernel<DK, DV, Tin, Tout>;
-    const int smem = ndir == 2 ? ReadSmem<DK, DV>::kBytes2 : ReadSmem<DK, DV>::kBytes1;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, ReadSmem<DK, DV>::kBytes2) !=
-        cudaSuccess)
+    constexpr int smem = ReadSmem<DK, DV>::kBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return GDN_ERR_CUDA;
     gdn::LaunchScope ls("vda_readout", a.stream);
     kern<<<dim3(a.F * ((a.U + 63) / 64), nbh), kThreads, smem, a.stream>>>(

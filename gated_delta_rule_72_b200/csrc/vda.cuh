@@ -119,18 +119,29 @@ vda_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const floa
 
 // ---------------------------------------------------------------------------
 // The frame chain of one head and direction.  Per frame (in the direction's
-// order): M = I + A_f, X = alpha_f S + B_f; M = L L^T (Cholesky, in place,
-// lower); L Y = X, L^T S' = Y.  The state each readout needs goes to `st`
+// order): M = I + A_f, X = alpha_f S + B_f; M = L L^T (Cholesky); L Y = X,
+// L^T S' = Y.  The state each readout needs goes to `st`
 // ([dir][F][B*H][DK][DV]): the causal direction stores S_f, the reverse one
 // R_{f+1} (before the frame is written).
+//
+// Cholesky, right-looking, one barrier per column: step j reads the pivot
+// and column j of the lower triangle, writes L's column j transposed into the
+// upper triangle (row j, which no later step reads or writes) and subtracts
+// the column's outer product from the trailing lower triangle; warp w takes
+// the rows i = w mod 16, its lanes the columns.  The diagonal of L goes to
+// its own array.  The triangular solves need no block barrier: each warp owns
+// 8 columns of X and each column's 4 lanes split its rows (i = g mod 4), so a
+// step only needs the column's own lanes, which share the warp.
 // ---------------------------------------------------------------------------
 template <int DK, int DV>
 struct ChainSmem {
     static constexpr int kLdM = DK + 1;                    // odd stride: column walks are conflict-free
+    static constexpr int kLdX = DV + 8;                    // 4 row groups of a column on 4 bank groups
     static constexpr int kM = 0;
     static constexpr int kS = kM + DK * kLdM * 4;          // state [DK][DV]
-    static constexpr int kX = kS + DK * DV * 4;            // right-hand side / solution [DK][DV]
-    static constexpr int kBytes = kX + DK * DV * 4;
+    static constexpr int kX = kS + DK * DV * 4;            // right-hand side / solution [DK][kLdX]
+    static constexpr int kD = kX + DK * kLdX * 4;          // diagonal of L, and its inverse
+    static constexpr int kBytes = kD + 2 * DK * 4;
 };
 
 template <int DK, int DV>
@@ -140,18 +151,25 @@ vda_chain_kernel(const float *__restrict__ A, const float *__restrict__ Bm, cons
                  float *__restrict__ st, int F, int H)
 {
     using SM = ChainSmem<DK, DV>;
-    constexpr int LD = SM::kLdM;
+    constexpr int LD = SM::kLdM, LX = SM::kLdX;
+    constexpr int NW = kChainThreads / 32;
+    static_assert(DV <= NW * 8, "8 columns of X per warp");
     extern __shared__ __align__(16) unsigned char csm[];
     float *M = reinterpret_cast<float *>(csm + SM::kM);
     float *S = reinterpret_cast<float *>(csm + SM::kS);
     float *X = reinterpret_cast<float *>(csm + SM::kX);
+    float *dL = reinterpret_cast<float *>(csm + SM::kD);
+    float *rdL = dL + DK;
     const int bh = blockIdx.x, nbh = gridDim.x, dir = blockIdx.y;
     const int b = bh / H, h = bh % H;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const float *src0 = dir ? s_in_bwd : s_in;   // (an output state may be its own input)
     float *dst_end = dir ? s_out_bwd : s_out;
     const size_t sdim = (size_t)DK * DV;
     for (int e = tid; e < DK * DV; e += kChainThreads) S[e] = src0 ? src0[bh * sdim + e] : 0.f;
+    // solve lanes: column c of X, row group g
+    const int c = warp * 8 + (lane & 7), g = lane >> 3;
+    const bool solver = c < DV;
 
     for (int step = 0; step < F; ++step) {
         const int f = dir ? F - 1 - step : step;
@@ -165,46 +183,50 @@ vda_chain_kernel(const float *__restrict__ A, const float *__restrict__ Bm, cons
             const int i = e / DK, j = e % DK;
             M[i * LD + j] = A[fh * DK * DK + e] + (i == j ? 1.f : 0.f);
         }
-        for (int e = tid; e < DK * DV; e += kChainThreads) X[e] = fmaf(a, S[e], Bm[fh * sdim + e]);
+        for (int e = tid; e < DK * DV; e += kChainThreads)
+            X[(e / DV) * LX + e % DV] = fmaf(a, S[e], Bm[fh * sdim + e]);
         __syncthreads();
-        // Cholesky, right-looking: column j scaled by 1/sqrt(pivot), then the
-        // trailing lower triangle loses the column's outer product
+        // ---- Cholesky
         for (int j = 0; j < DK; ++j) {
-            const float inv = rsqrtf(M[j * LD + j]);
-            __syncthreads();
-            for (int i = j + tid; i < DK; i += kChainThreads) M[i * LD + j] *= inv;
-            __syncthreads();
-            const int n = DK - 1 - j;
-            for (int e = tid; e < n * n; e += kChainThreads) {
-                const int i = j + 1 + e / n, c = j + 1 + e % n;
-                if (c <= i) M[i * LD + c] = fmaf(-M[i * LD + j], M[c * LD + j], M[i * LD + c]);
+            const float piv = M[j * LD + j];
+            const float r = rsqrtf(piv), r2 = r * r;
+            for (int i = j + 1 + ((warp - (j + 1)) & (NW - 1)); i < DK; i += NW) {
+                const float mij = M[i * LD + j];
+                if (lane == 0) M[j * LD + i] = mij * r;        // L[i][j], kept at (j, i)
+                const float fct = mij * r2;
+                for (int cc = j + 1 + lane; cc <= i; cc += 32)
+                    M[i * LD + cc] = fmaf(-fct, M[cc * LD + j], M[i * LD + cc]);
+            }
+            if (tid == 0) {
+                dL[j] = piv * r;
+                rdL[j] = r;
             }
             __syncthreads();
         }
-        // L Y = X (forward), then L^T S' = Y (backward), in place in X
-        for (int j = 0; j < DK; ++j) {
-            const float inv = 1.f / M[j * LD + j];
-            for (int c = tid; c < DV; c += kChainThreads) X[j * DV + c] *= inv;
-            __syncthreads();
-            for (int e = tid; e < (DK - 1 - j) * DV; e += kChainThreads) {
-                const int i = j + 1 + e / DV, c = e % DV;
-                X[i * DV + c] = fmaf(-M[i * LD + j], X[j * DV + c], X[i * DV + c]);
+        // ---- L Y = X, then L^T S' = Y, column by column inside each warp
+        if (solver) {
+            for (int j = 0; j < DK; ++j) {
+                const float y = X[j * LX + c] * rdL[j];
+                __syncwarp();
+                if ((j & 3) == g) X[j * LX + c] = y;
+                for (int i = j + 1 + ((g - (j + 1)) & 3); i < DK; i += 4)
+                    X[i * LX + c] = fmaf(-M[j * LD + i], y, X[i * LX + c]);   // L[i][j] at (j, i)
+                __syncwarp();
             }
-            __syncthreads();
-        }
-        for (int j = DK - 1; j >= 0; --j) {
-            const float inv = 1.f / M[j * LD + j];
-            for (int c = tid; c < DV; c += kChainThreads) X[j * DV + c] *= inv;
-            __syncthreads();
-            for (int e = tid; e < j * DV; e += kChainThreads) {
-                const int i = e / DV, c = e % DV;
-                X[i * DV + c] = fmaf(-M[j * LD + i], X[j * DV + c], X[i * DV + c]);
+            for (int j = DK - 1; j >= 0; --j) {
+                const float y = X[j * LX + c] * rdL[j];
+                __syncwarp();
+                if ((j & 3) == g) X[j * LX + c] = y;
+                for (int i = g; i < j; i += 4)
+                    X[i * LX + c] = fmaf(-M[i * LD + j], y, X[i * LX + c]);   // L[j][i] at (i, j)
+                __syncwarp();
             }
-            __syncthreads();
         }
+        __syncthreads();
         for (int e = tid; e < DK * DV; e += kChainThreads) {
-            S[e] = X[e];
-            if (!dir) dst[e] = X[e];
+            const float x = X[(e / DV) * LX + e % DV];
+            S[e] = x;
+            if (!dir) dst[e] = x;
         }
     }
     __syncthreads();
@@ -213,15 +235,15 @@ vda_chain_kernel(const float *__restrict__ A, const float *__restrict__ Bm, cons
 }
 
 // ---------------------------------------------------------------------------
-// Readout: 64 tokens of one frame per CTA, o = Q S (+ Q R).  Thread tile:
-// 4 tokens x 8 value columns (DV = 128; 4 columns for DV = 64).
+// Readout: 64 tokens of one frame per CTA, o = Q (S + R): the two directions'
+// states are added once while they are staged.  Thread tile: 4 tokens x 8
+// value columns (DV = 128; 4 columns for DV = 64).
 // ---------------------------------------------------------------------------
 template <int DK, int DV>
 struct ReadSmem {
     static constexpr int kQ = 0;                             // [DK][64] (transposed)
-    static constexpr int kS = kQ + DK * 64 * 4;              // [ndir][DK][DV]
-    static constexpr int kBytes1 = kS + DK * DV * 4;
-    static constexpr int kBytes2 = kS + 2 * DK * DV * 4;
+    static constexpr int kS = kQ + DK * 64 * 4;              // [DK][DV]
+    static constexpr int kBytes = kS + DK * DV * 4;
 };
 
 template <int DK, int DV, typename Tin, typename Tout>
@@ -244,9 +266,17 @@ vda_readout_kernel(const Tin *__restrict__ q, const float *__restrict__ st, Tout
         const int tk = e / DK, i = e % DK;
         Qt[i * 64 + tk] = tk < n ? to_f32(q[(((size_t)b * T + (size_t)f * U + u0 + tk) * H + h) * DK + i]) : 0.f;
     }
-    for (int d = 0; d < ndir; ++d) {
-        const float *src = st + ((size_t)d * F * nbh + (size_t)f * nbh + bh) * sdim;
-        for (int e = tid; e < DK * DV; e += kThreads) Ss[d * sdim + e] = src[e];
+    {
+        const float *s0 = st + ((size_t)f * nbh + bh) * sdim;
+        const float *s1 = s0 + (size_t)F * nbh * sdim;            // the reverse direction's
+        for (int e = tid * 4; e < DK * DV; e += kThreads * 4) {
+            float4 x = *reinterpret_cast<const float4 *>(s0 + e);
+            if (ndir == 2) {
+                const float4 y = *reinterpret_cast<const float4 *>(s1 + e);
+                x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+            }
+            *reinterpret_cast<float4 *>(Ss + e) = x;
+        }
     }
     __syncthreads();
     const int t0 = (tid / 16) * 4, c0 = (tid % 16) * TC;
@@ -255,8 +285,8 @@ vda_readout_kernel(const Tin *__restrict__ q, const float *__restrict__ st, Tout
     for (int r = 0; r < 4; ++r)
 #pragma unroll
         for (int c = 0; c < TC; ++c) acc[r][c] = 0.f;
-    for (int d = 0; d < ndir; ++d) {
-        const float *Sd = Ss + d * sdim;
+    {
+        const float *Sd = Ss;
 #pragma unroll 4
         for (int i = 0; i < DK; ++i) {
             const float4 qv = *reinterpret_cast<const float4 *>(Qt + i * 64 + t0);

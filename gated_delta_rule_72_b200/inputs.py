@@ -16,6 +16,9 @@ frame for the streaming rollout):
   bidir720   B=1, H=20, T=75,600, d=128, bf16  bidirectional
   rollout    B=1, H=16, 168 calls x 1,560 tokens, d=128, bf16, state carried
   skewed     B=4, H=32, T=16,384, d=128, bf16, fast-forgetting gates
+  vda480     B=1, H=12, T=32,760 = 21 frames x 1,560 tokens, d=128, bf16,
+             frame-wise delta operator, bidirectional (the per-frame decay is
+             the alpha drawn for the frame's first token)
 
 Distributions: q, k ~ N(0,1) then L2-normalised over the head dimension per
 token and head; v ~ N(0,1).  "default" gates: alpha = exp(-softplus(n)*0.05),
@@ -40,8 +43,9 @@ class Workload:
     dtype: str          # "f32" or "bf16": dtype of q, k, v and o
     seed: int
     gates: str = "default"
-    mode: str = "causal"  # "causal", "bidir" or "rollout"
+    mode: str = "causal"  # "causal", "bidir", "rollout" or "vda" (frame-wise, bidirectional)
     calls: int = 1        # rollout: number of successive calls of T tokens
+    frame: int = 0        # vda: tokens per frame
 
     @property
     def total_T(self) -> int:
@@ -58,7 +62,14 @@ WORKLOADS = {
     "bidir720": Workload("bidir720", 1, 75600, 20, 128, 128, "bf16", 2, mode="bidir"),
     "rollout": Workload("rollout", 1, 1560, 16, 128, 128, "bf16", 3, mode="rollout", calls=168),
     "skewed": Workload("skewed", 4, 16384, 32, 128, 128, "bf16", 4, gates="skewed"),
+    "vda480": Workload("vda480", 1, 32760, 12, 128, 128, "bf16", 5, mode="vda", frame=1560),
 }
+
+
+def frame_alpha(alpha: torch.Tensor, U: int) -> torch.Tensor:
+    """Per-frame decays [B, F, H] for frames of U tokens: the alpha drawn for
+    each frame's first token."""
+    return alpha[:, ::U].contiguous()
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
 
