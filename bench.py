@@ -88,13 +88,15 @@ def flops_per_token_head(w, C=64):
 
 def vda_kernel_flops(w):
     """FLOPs per token-head of the frame-wise operator's kernels (bidirectional):
-    the frame's key Gram and key-value products once, per direction a Cholesky
-    of I + A (dk^3/3), two triangular solves (2 dk^2 dv) and the right-hand
-    side (2 dk dv) per frame, and the readout (2 dk dv per token)."""
+    the frame's key Gram and key-value products (2 dk (dk + dv) per token);
+    per frame the Cholesky of I + A (dk^3/3) and the solves for P = (I + A)^-1
+    and C = P B (2 dk^2 (dk + dv)); per frame and direction S <- a P S + C
+    (2 dk^2 dv); the readout of the two summed states (2 dk dv per token)."""
     dk, dv, U = w.dk, w.dv, w.frame
     return {"vda_gram": 2.0 * dk * (dk + dv),
-            "vda_chain": 2 * (dk ** 3 / 3.0 + 2.0 * dk * dk * dv + 2.0 * dk * dv) / U,
-            "vda_readout": 2 * 2.0 * dk * dv}
+            "vda_factor": (dk ** 3 / 3.0 + 2.0 * dk * dk * (dk + dv)) / U,
+            "vda_chain": 2 * 2.0 * dk * dk * dv / U,
+            "vda_readout": 2.0 * dk * dv}
 
 
 # fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA/clk x 2 FLOP x 1.965 GHz

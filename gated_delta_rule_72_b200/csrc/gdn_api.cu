@@ -613,6 +613,15 @@ gdn_status run_vda(const VdaArgs &a) {
         if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
     }
     {
+        auto kern = vda_factor_kernel<DK, DV>;
+        constexpr int smem = FactorSmem<DK, DV>::kBytes;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        gdn::LaunchScope ls("vda_factor", a.stream);
+        kern<<<dim3(a.F, nbh), kChainThreads, smem, a.stream>>>(A, Bm);
+        if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
+    }
+    {
         auto kern = vda_chain_kernel<DK, DV>;
         constexpr int smem = ChainSmem<DK, DV>::kBytes;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)

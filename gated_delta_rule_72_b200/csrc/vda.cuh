@@ -11,12 +11,15 @@
 // f: o_u = S_f^T q_u (+ R_{f+1}^T q_u for a bidirectional scan: the frames
 // after f only).
 //
-// Three kernels:
+// Four kernels:
 //   vda_gram    (frame x head, fully parallel)  A_f and B_f
-//   vda_chain   (head x direction, sequential over frames)  Cholesky of
-//               I + A_f and two triangular solves per frame, the state in
-//               shared memory; stores the state each frame's readout uses
-//   vda_readout (token block x head, fully parallel)  o = Q S (+ Q R)
+//   vda_factor  (frame x head, fully parallel)  P_f = (I + A_f)^{-1} and
+//               C_f = P_f B_f by a Cholesky factorisation: none of it depends
+//               on the state
+//   vda_chain   (head x direction, sequential over frames)  S <- alpha_f P_f S
+//               + C_f, the state in shared memory; stores the state each
+//               frame's readout uses
+//   vda_readout (token block x head, fully parallel)  o = Q (S + R)
 #pragma once
 
 #include "common.cuh"
@@ -118,115 +121,178 @@ vda_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const floa
 }
 
 // ---------------------------------------------------------------------------
-// The frame chain of one head and direction.  Per frame (in the direction's
-// order): M = I + A_f, X = alpha_f S + B_f; M = L L^T (Cholesky); L Y = X,
-// L^T S' = Y.  The state each readout needs goes to `st`
-// ([dir][F][B*H][DK][DV]): the causal direction stores S_f, the reverse one
-// R_{f+1} (before the frame is written).
+// Factor (frame x head, fully parallel: nothing here depends on the state):
+// P_f = (I + A_f)^{-1} and C_f = P_f B_f, written over A_f and B_f.
 //
-// Cholesky, right-looking, one barrier per column: step j reads the pivot
-// and column j of the lower triangle, writes L's column j transposed into the
-// upper triangle (row j, which no later step reads or writes) and subtracts
-// the column's outer product from the trailing lower triangle; warp w takes
-// the rows i = w mod 16, its lanes the columns.  The diagonal of L goes to
-// its own array.  The triangular solves need no block barrier: each warp owns
-// 8 columns of X and each column's 4 lanes split its rows (i = g mod 4), so a
-// step only needs the column's own lanes, which share the warp.
+// M = I + A_f = L L^T (Cholesky, right-looking, one barrier per column: step
+// j reads the pivot and column j of the lower triangle, writes L's column j
+// transposed into the upper triangle (row j, which no later step reads or
+// writes) and subtracts the column's outer product from the trailing lower
+// triangle; warp w takes the rows i = w mod 16, its lanes the columns).
+// Then L Y = [I | B_f] and L^T [P | C] = Y with no block barrier: each warp
+// owns 8 right-hand-side columns at a time, each column's 4 lanes split its
+// rows (i = g mod 4), so a step only involves lanes of one warp.
 // ---------------------------------------------------------------------------
 template <int DK, int DV>
-struct ChainSmem {
+struct FactorSmem {
+    static constexpr int kW = DK + DV;                     // right-hand sides [I | B]
     static constexpr int kLdM = DK + 1;                    // odd stride: column walks are conflict-free
-    static constexpr int kLdX = DV + 8;                    // 4 row groups of a column on 4 bank groups
+    static constexpr int kLdX = kW + 8;                    // 4 row groups of a column on 4 bank groups
     static constexpr int kM = 0;
-    static constexpr int kS = kM + DK * kLdM * 4;          // state [DK][DV]
-    static constexpr int kX = kS + DK * DV * 4;            // right-hand side / solution [DK][kLdX]
-    static constexpr int kD = kX + DK * kLdX * 4;          // diagonal of L, and its inverse
-    static constexpr int kBytes = kD + 2 * DK * 4;
+    static constexpr int kX = kM + DK * kLdM * 4;
+    static constexpr int kD = kX + DK * kLdX * 4;          // 1 / diagonal of L
+    static constexpr int kBytes = kD + DK * 4;
 };
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kChainThreads)
-vda_chain_kernel(const float *__restrict__ A, const float *__restrict__ Bm, const float *__restrict__ alpha_f,
+vda_factor_kernel(float *__restrict__ A, float *__restrict__ Bm)
+{
+    using SM = FactorSmem<DK, DV>;
+    constexpr int LD = SM::kLdM, LX = SM::kLdX, W = SM::kW;
+    constexpr int NW = kChainThreads / 32;
+    static_assert(W % 8 == 0, "right-hand-side columns in groups of 8 (warp-uniform loop bounds)");
+    extern __shared__ __align__(16) unsigned char fsm[];
+    float *M = reinterpret_cast<float *>(fsm + SM::kM);
+    float *X = reinterpret_cast<float *>(fsm + SM::kX);
+    float *rdL = reinterpret_cast<float *>(fsm + SM::kD);
+    const size_t fh = (size_t)blockIdx.x * gridDim.y + blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float *Af = A + fh * DK * DK, *Bf = Bm + fh * DK * DV;
+    for (int e = tid; e < DK * DK; e += kChainThreads) {
+        const int i = e / DK, j = e % DK;
+        M[i * LD + j] = Af[e] + (i == j ? 1.f : 0.f);
+        X[i * LX + j] = i == j ? 1.f : 0.f;
+    }
+    for (int e = tid; e < DK * DV; e += kChainThreads) X[(e / DV) * LX + DK + e % DV] = Bf[e];
+    __syncthreads();
+    // ---- Cholesky
+    for (int j = 0; j < DK; ++j) {
+        const float piv = M[j * LD + j];
+        const float r = rsqrtf(piv), r2 = r * r;
+        for (int i = j + 1 + ((warp - (j + 1)) & (NW - 1)); i < DK; i += NW) {
+            const float mij = M[i * LD + j];
+            if (lane == 0) M[j * LD + i] = mij * r;        // L[i][j], kept at (j, i)
+            const float fct = mij * r2;
+            for (int cc = j + 1 + lane; cc <= i; cc += 32)
+                M[i * LD + cc] = fmaf(-fct, M[cc * LD + j], M[i * LD + cc]);
+        }
+        if (tid == 0) rdL[j] = r;                          // 1 / L[j][j]
+        __syncthreads();
+    }
+    // ---- L Y = [I | B], then L^T [P | C] = Y, column by column inside each warp
+    const int g = lane >> 3;
+    for (int c = warp * 8 + (lane & 7); c < W; c += NW * 8) {
+        for (int j = 0; j < DK; ++j) {
+            const float y = X[j * LX + c] * rdL[j];
+            __syncwarp();
+            if ((j & 3) == g) X[j * LX + c] = y;
+            for (int i = j + 1 + ((g - (j + 1)) & 3); i < DK; i += 4)
+                X[i * LX + c] = fmaf(-M[j * LD + i], y, X[i * LX + c]);   // L[i][j] at (j, i)
+            __syncwarp();
+        }
+        for (int j = DK - 1; j >= 0; --j) {
+            const float y = X[j * LX + c] * rdL[j];
+            __syncwarp();
+            if ((j & 3) == g) X[j * LX + c] = y;
+            for (int i = g; i < j; i += 4)
+                X[i * LX + c] = fmaf(-M[i * LD + j], y, X[i * LX + c]);   // L[j][i] at (i, j)
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < DK * DK; e += kChainThreads) Af[e] = X[(e / DK) * LX + e % DK];
+    for (int e = tid; e < DK * DV; e += kChainThreads) Bf[e] = X[(e / DV) * LX + DK + e % DV];
+}
+
+// ---------------------------------------------------------------------------
+// The frame chain of one head and direction: S <- alpha_f P_f S + C_f per
+// frame, in the direction's order.  The state each readout needs goes to
+// `st` ([dir][F][B*H][DK][DV]): the causal direction stores S_f, the reverse
+// one R_{f+1} (before the frame is written).  Thread tile 4 rows x 8 columns
+// of S (DK x DV over 512 threads); P_f (symmetric: row k of P is column k) is
+// staged in shared memory.
+// ---------------------------------------------------------------------------
+template <int DK, int DV>
+struct ChainSmem {
+    static constexpr int kP = 0;                           // [DK][DK]
+    static constexpr int kS = kP + DK * DK * 4;            // [DK][DV]
+    static constexpr int kBytes = kS + DK * DV * 4;
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kChainThreads)
+vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ C, const float *__restrict__ alpha_f,
                  const float *s_in, const float *s_in_bwd, float *s_out, float *s_out_bwd,
                  float *__restrict__ st, int F, int H)
 {
     using SM = ChainSmem<DK, DV>;
-    constexpr int LD = SM::kLdM, LX = SM::kLdX;
-    constexpr int NW = kChainThreads / 32;
-    static_assert(DV <= NW * 8, "8 columns of X per warp");
+    constexpr int TR = 4, TCc = 8;
+    constexpr int NCT = DV / TCc;                      // column tiles
+    constexpr int kTiles = (DK / TR) * NCT;
+    static_assert(kTiles <= kChainThreads, "thread tiles");
     extern __shared__ __align__(16) unsigned char csm[];
-    float *M = reinterpret_cast<float *>(csm + SM::kM);
+    float *Ps = reinterpret_cast<float *>(csm + SM::kP);
     float *S = reinterpret_cast<float *>(csm + SM::kS);
-    float *X = reinterpret_cast<float *>(csm + SM::kX);
-    float *dL = reinterpret_cast<float *>(csm + SM::kD);
-    float *rdL = dL + DK;
     const int bh = blockIdx.x, nbh = gridDim.x, dir = blockIdx.y;
     const int b = bh / H, h = bh % H;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x;
     const float *src0 = dir ? s_in_bwd : s_in;   // (an output state may be its own input)
     float *dst_end = dir ? s_out_bwd : s_out;
     const size_t sdim = (size_t)DK * DV;
     for (int e = tid; e < DK * DV; e += kChainThreads) S[e] = src0 ? src0[bh * sdim + e] : 0.f;
-    // solve lanes: column c of X, row group g
-    const int c = warp * 8 + (lane & 7), g = lane >> 3;
-    const bool solver = c < DV;
+    const bool worker = tid < kTiles;
+    const int i0 = (tid / NCT) * TR, c0 = (tid % NCT) * TCc;
 
     for (int step = 0; step < F; ++step) {
         const int f = dir ? F - 1 - step : step;
         const size_t fh = (size_t)f * nbh + bh;
         const float a = alpha_f[((size_t)b * F + f) * H + h];
-        __syncthreads();
         float *dst = st + ((size_t)dir * F * nbh + fh) * sdim;
+        __syncthreads();                                   // S complete, P free
         if (dir)   // the reverse readout of frame f reads R_{f+1}
-            for (int e = tid; e < DK * DV; e += kChainThreads) dst[e] = S[e];
-        for (int e = tid; e < DK * DK; e += kChainThreads) {
-            const int i = e / DK, j = e % DK;
-            M[i * LD + j] = A[fh * DK * DK + e] + (i == j ? 1.f : 0.f);
-        }
-        for (int e = tid; e < DK * DV; e += kChainThreads)
-            X[(e / DV) * LX + e % DV] = fmaf(a, S[e], Bm[fh * sdim + e]);
+            for (int e = tid * 4; e < DK * DV; e += kChainThreads * 4)
+                *reinterpret_cast<float4 *>(dst + e) = *reinterpret_cast<const float4 *>(S + e);
+        for (int e = tid * 4; e < DK * DK; e += kChainThreads * 4)
+            *reinterpret_cast<float4 *>(Ps + e) = *reinterpret_cast<const float4 *>(P + fh * DK * DK + e);
         __syncthreads();
-        // ---- Cholesky
-        for (int j = 0; j < DK; ++j) {
-            const float piv = M[j * LD + j];
-            const float r = rsqrtf(piv), r2 = r * r;
-            for (int i = j + 1 + ((warp - (j + 1)) & (NW - 1)); i < DK; i += NW) {
-                const float mij = M[i * LD + j];
-                if (lane == 0) M[j * LD + i] = mij * r;        // L[i][j], kept at (j, i)
-                const float fct = mij * r2;
-                for (int cc = j + 1 + lane; cc <= i; cc += 32)
-                    M[i * LD + cc] = fmaf(-fct, M[cc * LD + j], M[i * LD + cc]);
-            }
-            if (tid == 0) {
-                dL[j] = piv * r;
-                rdL[j] = r;
-            }
-            __syncthreads();
-        }
-        // ---- L Y = X, then L^T S' = Y, column by column inside each warp
-        if (solver) {
-            for (int j = 0; j < DK; ++j) {
-                const float y = X[j * LX + c] * rdL[j];
-                __syncwarp();
-                if ((j & 3) == g) X[j * LX + c] = y;
-                for (int i = j + 1 + ((g - (j + 1)) & 3); i < DK; i += 4)
-                    X[i * LX + c] = fmaf(-M[j * LD + i], y, X[i * LX + c]);   // L[i][j] at (j, i)
-                __syncwarp();
-            }
-            for (int j = DK - 1; j >= 0; --j) {
-                const float y = X[j * LX + c] * rdL[j];
-                __syncwarp();
-                if ((j & 3) == g) X[j * LX + c] = y;
-                for (int i = g; i < j; i += 4)
-                    X[i * LX + c] = fmaf(-M[i * LD + j], y, X[i * LX + c]);   // L[j][i] at (i, j)
-                __syncwarp();
+        float acc[TR][TCc];
+        if (worker) {
+#pragma unroll
+            for (int r = 0; r < TR; ++r)
+#pragma unroll
+                for (int cc = 0; cc < TCc; ++cc) acc[r][cc] = 0.f;
+#pragma unroll 4
+            for (int kk = 0; kk < DK; ++kk) {
+                const float4 pv = *reinterpret_cast<const float4 *>(Ps + kk * DK + i0);   // P[i0..][kk]
+                const float pa[TR] = {pv.x, pv.y, pv.z, pv.w};
+                const float4 s0 = *reinterpret_cast<const float4 *>(S + kk * DV + c0);
+                const float4 s1 = *reinterpret_cast<const float4 *>(S + kk * DV + c0 + 4);
+                const float sv[TCc] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+                for (int r = 0; r < TR; ++r)
+#pragma unroll
+                    for (int cc = 0; cc < TCc; ++cc) acc[r][cc] = fmaf(pa[r], sv[cc], acc[r][cc]);
             }
         }
-        __syncthreads();
-        for (int e = tid; e < DK * DV; e += kChainThreads) {
-            const float x = X[(e / DV) * LX + e % DV];
-            S[e] = x;
-            if (!dir) dst[e] = x;
+        __syncthreads();                                   // every read of the old S is done
+        if (worker) {
+#pragma unroll
+            for (int r = 0; r < TR; ++r) {
+                const size_t row = (size_t)(i0 + r) * DV + c0;
+                const float4 c0v = *reinterpret_cast<const float4 *>(C + fh * sdim + row);
+                const float4 c1v = *reinterpret_cast<const float4 *>(C + fh * sdim + row + 4);
+                const float4 n0 = make_float4(fmaf(a, acc[r][0], c0v.x), fmaf(a, acc[r][1], c0v.y),
+                                              fmaf(a, acc[r][2], c0v.z), fmaf(a, acc[r][3], c0v.w));
+                const float4 n1 = make_float4(fmaf(a, acc[r][4], c1v.x), fmaf(a, acc[r][5], c1v.y),
+                                              fmaf(a, acc[r][6], c1v.z), fmaf(a, acc[r][7], c1v.w));
+                *reinterpret_cast<float4 *>(S + row) = n0;
+                *reinterpret_cast<float4 *>(S + row + 4) = n1;
+                if (!dir) {
+                    *reinterpret_cast<float4 *>(dst + row) = n0;
+                    *reinterpret_cast<float4 *>(dst + row + 4) = n1;
+                }
+            }
         }
     }
     __syncthreads();
