@@ -20,6 +20,7 @@
 #include "readout.cuh"
 #include "token_step.cuh"
 #include "vda.cuh"
+#include "vda_tc.cuh"
 
 // Count of bounded device-side waits that gave up (see gdn_device_timeouts).
 static __device__ unsigned int g_wait_timeouts;
@@ -602,7 +603,22 @@ gdn_status run_vda(const VdaArgs &a) {
     float *A = static_cast<float *>(a.ws);
     float *Bm = reinterpret_cast<float *>(static_cast<char *>(a.ws) + round_up(fh * DK * DK * 4, 256));
     float *st = reinterpret_cast<float *>(reinterpret_cast<char *>(Bm) + round_up(fh * DK * DV * 4, 256));
-    {
+    if (std::is_same<Tin, __nv_bfloat16>::value && DK == 128) {
+        // bf16 keys and values: the Gram and key-value products on the tensor cores
+        CUtensorMap mk, mv;
+        if (!encode_map(&mk, a.k, a.B, a.F * a.U, a.H, DK, 64, 128) ||
+            !encode_map(&mv, a.v, a.B, a.F * a.U, a.H, DV, 64, 128))
+            return GDN_ERR_CUDA;
+        unsigned int *err = timeout_counter();
+        if (!err) return GDN_ERR_CUDA;
+        auto kern = vda_gram_tc_kernel<DV>;
+        constexpr int smem = GramTcSmem<DV>::kAlloc;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        gdn::LaunchScope ls("vda_gram_tc", a.stream);
+        kern<<<dim3(a.F, nbh), kTcThreads, smem, a.stream>>>(mk, mv, a.beta, A, Bm, a.F, a.U, a.H, err);
+        if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
+    } else {
         auto kern = vda_gram_kernel<DK, DV, Tin>;
         constexpr int smem = GramSmem<DK, DV>::kBytes;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -621,8 +637,9 @@ gdn_status run_vda(const VdaArgs &a) {
         kern<<<dim3(a.F, nbh), kChainThreads, smem, a.stream>>>(A, Bm);
         if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
     }
+    constexpr bool kTc = std::is_same<Tin, __nv_bfloat16>::value && DK == 128;
     {
-        auto kern = vda_chain_kernel<DK, DV>;
+        auto kern = vda_chain_kernel<DK, DV, kTc>;
         constexpr int smem = ChainSmem<DK, DV>::kBytes;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return GDN_ERR_CUDA;
@@ -630,6 +647,20 @@ gdn_status run_vda(const VdaArgs &a) {
         kern<<<dim3(nbh, ndir), kChainThreads, smem, a.stream>>>(A, Bm, a.alpha_f, a.s_in, a.s_in_bwd, a.s_out,
                                                                 a.s_out_bwd, st, a.F, a.H);
         if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
+    }
+    if (kTc) {   // states as operand images: the readout on the tensor cores
+        CUtensorMap mq;
+        if (!encode_map(&mq, a.q, a.B, a.F * a.U, a.H, DK, 64, 128)) return GDN_ERR_CUDA;
+        unsigned int *err = timeout_counter();
+        if (!err) return GDN_ERR_CUDA;
+        auto kern = vda_readout_tc_kernel<DV, Tout>;
+        constexpr int smem = ReadTcSmem<DV>::kAlloc;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return GDN_ERR_CUDA;
+        gdn::LaunchScope ls("vda_readout_tc", a.stream);
+        kern<<<dim3(a.F * ((a.U + 127) / 128), nbh), 128, smem, a.stream>>>(
+            mq, reinterpret_cast<const unsigned char *>(st), static_cast<Tout *>(a.o), a.F, a.U, a.H, ndir, err);
+        return launch_status();
     }
     auto kern = vda_readout_kernel<DK, DV, Tin, Tout>;
     constexpr int smem = ReadSmem<DK, DV>::kBytes;

@@ -174,29 +174,53 @@ vda_factor_kernel(float *__restrict__ A, float *__restrict__ Bm)
             const float mij = M[i * LD + j];
             if (lane == 0) M[j * LD + i] = mij * r;        // L[i][j], kept at (j, i)
             const float fct = mij * r2;
-            for (int cc = j + 1 + lane; cc <= i; cc += 32)
-                M[i * LD + cc] = fmaf(-fct, M[cc * LD + j], M[i * LD + cc]);
+            int cc = j + 1 + lane;
+            for (; cc + 96 <= i; cc += 128) {              // four columns loaded before any store
+                float lc[4], m[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    lc[q] = M[(cc + 32 * q) * LD + j];
+                    m[q] = M[i * LD + cc + 32 * q];
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) M[i * LD + cc + 32 * q] = fmaf(-fct, lc[q], m[q]);
+            }
+            for (; cc <= i; cc += 32) M[i * LD + cc] = fmaf(-fct, M[cc * LD + j], M[i * LD + cc]);
         }
         if (tid == 0) rdL[j] = r;                          // 1 / L[j][j]
         __syncthreads();
     }
-    // ---- L Y = [I | B], then L^T [P | C] = Y, column by column inside each warp
+    // ---- L Y = [I | B], then L^T [P | C] = Y, column by column inside each warp.
+    // A step's row updates are independent: four rows are loaded before any is
+    // stored, so their shared-memory latencies overlap.
     const int g = lane >> 3;
+    auto update_rows = [&](int i, int i_end, int c, float y, int lstride, int loff) {
+        // X[i][c] -= L * y for rows i, i+4, ... < i_end; L of row i at M[i*lstride + loff]
+        for (; i + 12 < i_end; i += 16) {
+            float l[4], x[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                l[q] = M[(i + 4 * q) * lstride + loff];
+                x[q] = X[(i + 4 * q) * LX + c];
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) X[(i + 4 * q) * LX + c] = fmaf(-l[q], y, x[q]);
+        }
+        for (; i < i_end; i += 4) X[i * LX + c] = fmaf(-M[i * lstride + loff], y, X[i * LX + c]);
+    };
     for (int c = warp * 8 + (lane & 7); c < W; c += NW * 8) {
         for (int j = 0; j < DK; ++j) {
             const float y = X[j * LX + c] * rdL[j];
             __syncwarp();
             if ((j & 3) == g) X[j * LX + c] = y;
-            for (int i = j + 1 + ((g - (j + 1)) & 3); i < DK; i += 4)
-                X[i * LX + c] = fmaf(-M[j * LD + i], y, X[i * LX + c]);   // L[i][j] at (j, i)
+            update_rows(j + 1 + ((g - (j + 1)) & 3), DK, c, y, 1, j * LD);    // L[i][j] at (j, i)
             __syncwarp();
         }
         for (int j = DK - 1; j >= 0; --j) {
             const float y = X[j * LX + c] * rdL[j];
             __syncwarp();
             if ((j & 3) == g) X[j * LX + c] = y;
-            for (int i = g; i < j; i += 4)
-                X[i * LX + c] = fmaf(-M[i * LD + j], y, X[i * LX + c]);   // L[j][i] at (i, j)
+            update_rows(g, j, c, y, LD, j);                                   // L[j][i] at (i, j)
             __syncwarp();
         }
     }
@@ -213,6 +237,30 @@ vda_factor_kernel(float *__restrict__ A, float *__restrict__ Bm)
 // of S (DK x DV over 512 threads); P_f (symmetric: row k of P is column k) is
 // staged in shared memory.
 // ---------------------------------------------------------------------------
+// State image for the tensor-core readout: [S_hi | S_lo] as bf16, the
+// operand layout of a 128B-swizzled MN-major B tile (rows = the key index,
+// groups of 64 columns 16 KB apart); S_hi + S_lo = S to about 2^-16.  Same
+// byte size as the fp32 state.
+__device__ __forceinline__ int img_off(int i, int n) {
+    const int L = i * 128 + (n & 63) * 2;
+    return (n >> 6) * 16384 + (L ^ (((L >> 7) & 7) << 4));
+}
+template <int DV>
+__device__ __forceinline__ void store_image_row8(unsigned char *img, int i, int n, const float *x) {
+    uint4 hi, lo;
+    uint32_t *ph = reinterpret_cast<uint32_t *>(&hi), *pl = reinterpret_cast<uint32_t *>(&lo);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+        const float2 hf = __bfloat1622float2(hv);
+        const __nv_bfloat162 lv = __floats2bfloat162_rn(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
+        ph[q] = *reinterpret_cast<const uint32_t *>(&hv);
+        pl[q] = *reinterpret_cast<const uint32_t *>(&lv);
+    }
+    *reinterpret_cast<uint4 *>(img + img_off(i, n)) = hi;
+    *reinterpret_cast<uint4 *>(img + img_off(i, n + DV)) = lo;
+}
+
 template <int DK, int DV>
 struct ChainSmem {
     static constexpr int kP = 0;                           // [DK][DK]
@@ -220,7 +268,9 @@ struct ChainSmem {
     static constexpr int kBytes = kS + DK * DV * 4;
 };
 
-template <int DK, int DV>
+// kImage: the states for the readout are stored as tensor-core operand images
+// (store_image_row8) instead of fp32.
+template <int DK, int DV, bool kImage>
 __global__ void __launch_bounds__(kChainThreads)
 vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ C, const float *__restrict__ alpha_f,
                  const float *s_in, const float *s_in_bwd, float *s_out, float *s_out_bwd,
@@ -250,9 +300,18 @@ vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ C, const
         const float a = alpha_f[((size_t)b * F + f) * H + h];
         float *dst = st + ((size_t)dir * F * nbh + fh) * sdim;
         __syncthreads();                                   // S complete, P free
-        if (dir)   // the reverse readout of frame f reads R_{f+1}
-            for (int e = tid * 4; e < DK * DV; e += kChainThreads * 4)
-                *reinterpret_cast<float4 *>(dst + e) = *reinterpret_cast<const float4 *>(S + e);
+        if (dir) {   // the reverse readout of frame f reads R_{f+1}
+            if (kImage) {
+                if (worker)
+#pragma unroll
+                    for (int r = 0; r < TR; ++r)
+                        store_image_row8<DV>(reinterpret_cast<unsigned char *>(dst), i0 + r, c0,
+                                             S + (i0 + r) * DV + c0);
+            } else {
+                for (int e = tid * 4; e < DK * DV; e += kChainThreads * 4)
+                    *reinterpret_cast<float4 *>(dst + e) = *reinterpret_cast<const float4 *>(S + e);
+            }
+        }
         for (int e = tid * 4; e < DK * DK; e += kChainThreads * 4)
             *reinterpret_cast<float4 *>(Ps + e) = *reinterpret_cast<const float4 *>(P + fh * DK * DK + e);
         __syncthreads();
@@ -289,8 +348,13 @@ vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ C, const
                 *reinterpret_cast<float4 *>(S + row) = n0;
                 *reinterpret_cast<float4 *>(S + row + 4) = n1;
                 if (!dir) {
-                    *reinterpret_cast<float4 *>(dst + row) = n0;
-                    *reinterpret_cast<float4 *>(dst + row + 4) = n1;
+                    if (kImage) {
+                        const float x8[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+                        store_image_row8<DV>(reinterpret_cast<unsigned char *>(dst), i0 + r, c0, x8);
+                    } else {
+                        *reinterpret_cast<float4 *>(dst + row) = n0;
+                        *reinterpret_cast<float4 *>(dst + row + 4) = n1;
+                    }
                 }
             }
         }
