@@ -90,11 +90,11 @@ def vda_kernel_flops(w):
     """FLOPs per token-head of the frame-wise operator's kernels (bidirectional):
     the frame's key Gram and key-value products (2 dk (dk + dv) per token);
     per frame the Cholesky of I + A (dk^3/3) and the solves for P = (I + A)^-1
-    and C = P B (2 dk^2 (dk + dv)); per frame and direction S <- a P S + C
-    (2 dk^2 dv); the readout of the two summed states (2 dk dv per token)."""
+    (2 dk^3); per frame and direction S <- P (a S + B) (2 dk^2 dv); the
+    readout of the two summed states (2 dk dv per token)."""
     dk, dv, U = w.dk, w.dv, w.frame
     return {"vda_gram": 2.0 * dk * (dk + dv),
-            "vda_factor": (dk ** 3 / 3.0 + 2.0 * dk * dk * (dk + dv)) / U,
+            "vda_factor": (dk ** 3 / 3.0 + 2.0 * dk ** 3) / U,
             "vda_chain": 2 * 2.0 * dk * dk * dv / U,
             "vda_readout": 2.0 * dk * dv}
 

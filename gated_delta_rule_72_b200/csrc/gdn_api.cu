@@ -634,7 +634,7 @@ gdn_status run_vda(const VdaArgs &a) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return GDN_ERR_CUDA;
         gdn::LaunchScope ls("vda_factor", a.stream);
-        kern<<<dim3(a.F, nbh), kChainThreads, smem, a.stream>>>(A, Bm);
+        kern<<<dim3(a.F, nbh), kChainThreads, smem, a.stream>>>(A);
         if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
     }
     constexpr bool kTc = std::is_same<Tin, __nv_bfloat16>::value && DK == 128;

@@ -13,11 +13,10 @@
 //
 // Four kernels:
 //   vda_gram    (frame x head, fully parallel)  A_f and B_f
-//   vda_factor  (frame x head, fully parallel)  P_f = (I + A_f)^{-1} and
-//               C_f = P_f B_f by a Cholesky factorisation: none of it depends
-//               on the state
-//   vda_chain   (head x direction, sequential over frames)  S <- alpha_f P_f S
-//               + C_f, the state in shared memory; stores the state each
+//   vda_factor  (frame x head, fully parallel)  P_f = (I + A_f)^{-1} by a
+//               Cholesky factorisation: none of it depends on the state
+//   vda_chain   (head x direction, sequential over frames)  S <- P_f (alpha_f S
+//               + B_f), the state in shared memory; stores the state each
 //               frame's readout uses
 //   vda_readout (token block x head, fully parallel)  o = Q (S + R)
 #pragma once
@@ -122,20 +121,20 @@ vda_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const floa
 
 // ---------------------------------------------------------------------------
 // Factor (frame x head, fully parallel: nothing here depends on the state):
-// P_f = (I + A_f)^{-1} and C_f = P_f B_f, written over A_f and B_f.
+// P_f = (I + A_f)^{-1}, written over A_f.
 //
 // M = I + A_f = L L^T (Cholesky, right-looking, one barrier per column: step
 // j reads the pivot and column j of the lower triangle, writes L's column j
 // transposed into the upper triangle (row j, which no later step reads or
 // writes) and subtracts the column's outer product from the trailing lower
 // triangle; warp w takes the rows i = w mod 16, its lanes the columns).
-// Then L Y = [I | B_f] and L^T [P | C] = Y with no block barrier: each warp
-// owns 8 right-hand-side columns at a time, each column's 4 lanes split its
-// rows (i = g mod 4), so a step only involves lanes of one warp.
+// Then L Y = I and L^T P = Y with no block barrier: each warp owns 8
+// right-hand-side columns, each column's 4 lanes split its rows (i = g mod
+// 4), so a step only involves lanes of one warp.
 // ---------------------------------------------------------------------------
 template <int DK, int DV>
 struct FactorSmem {
-    static constexpr int kW = DK + DV;                     // right-hand sides [I | B]
+    static constexpr int kW = DK;                          // right-hand sides: I
     static constexpr int kLdM = DK + 1;                    // odd stride: column walks are conflict-free
     static constexpr int kLdX = kW + 8;                    // 4 row groups of a column on 4 bank groups
     static constexpr int kM = 0;
@@ -146,7 +145,7 @@ struct FactorSmem {
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kChainThreads)
-vda_factor_kernel(float *__restrict__ A, float *__restrict__ Bm)
+vda_factor_kernel(float *__restrict__ A)
 {
     using SM = FactorSmem<DK, DV>;
     constexpr int LD = SM::kLdM, LX = SM::kLdX, W = SM::kW;
@@ -158,13 +157,12 @@ vda_factor_kernel(float *__restrict__ A, float *__restrict__ Bm)
     float *rdL = reinterpret_cast<float *>(fsm + SM::kD);
     const size_t fh = (size_t)blockIdx.x * gridDim.y + blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    float *Af = A + fh * DK * DK, *Bf = Bm + fh * DK * DV;
+    float *Af = A + fh * DK * DK;
     for (int e = tid; e < DK * DK; e += kChainThreads) {
         const int i = e / DK, j = e % DK;
         M[i * LD + j] = Af[e] + (i == j ? 1.f : 0.f);
         X[i * LX + j] = i == j ? 1.f : 0.f;
     }
-    for (int e = tid; e < DK * DV; e += kChainThreads) X[(e / DV) * LX + DK + e % DV] = Bf[e];
     __syncthreads();
     // ---- Cholesky
     for (int j = 0; j < DK; ++j) {
@@ -190,7 +188,7 @@ vda_factor_kernel(float *__restrict__ A, float *__restrict__ Bm)
         if (tid == 0) rdL[j] = r;                          // 1 / L[j][j]
         __syncthreads();
     }
-    // ---- L Y = [I | B], then L^T [P | C] = Y, column by column inside each warp.
+    // ---- L Y = I, then L^T P = Y, column by column inside each warp.
     // A step's row updates are independent: four rows are loaded before any is
     // stored, so their shared-memory latencies overlap.
     const int g = lane >> 3;
@@ -226,11 +224,10 @@ vda_factor_kernel(float *__restrict__ A, float *__restrict__ Bm)
     }
     __syncthreads();
     for (int e = tid; e < DK * DK; e += kChainThreads) Af[e] = X[(e / DK) * LX + e % DK];
-    for (int e = tid; e < DK * DV; e += kChainThreads) Bf[e] = X[(e / DV) * LX + DK + e % DV];
 }
 
 // ---------------------------------------------------------------------------
-// The frame chain of one head and direction: S <- alpha_f P_f S + C_f per
+// The frame chain of one head and direction: S <- P_f (alpha_f S + B_f) per
 // frame, in the direction's order.  The state each readout needs goes to
 // `st` ([dir][F][B*H][DK][DV]): the causal direction stores S_f, the reverse
 // one R_{f+1} (before the frame is written).  Thread tile 4 rows x 8 columns
@@ -272,7 +269,7 @@ struct ChainSmem {
 // (store_image_row8) instead of fp32.
 template <int DK, int DV, bool kImage>
 __global__ void __launch_bounds__(kChainThreads)
-vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ C, const float *__restrict__ alpha_f,
+vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ Bm, const float *__restrict__ alpha_f,
                  const float *s_in, const float *s_in_bwd, float *s_out, float *s_out_bwd,
                  float *__restrict__ st, int F, int H)
 {
@@ -314,6 +311,13 @@ vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ C, const
         }
         for (int e = tid * 4; e < DK * DK; e += kChainThreads * 4)
             *reinterpret_cast<float4 *>(Ps + e) = *reinterpret_cast<const float4 *>(P + fh * DK * DK + e);
+        __syncthreads();   // (the reverse direction's store above has read S)
+        for (int e = tid * 4; e < DK * DV; e += kChainThreads * 4) {   // S <- alpha S + B
+            float4 x = *reinterpret_cast<const float4 *>(S + e);
+            const float4 bb = *reinterpret_cast<const float4 *>(Bm + fh * sdim + e);
+            x.x = fmaf(a, x.x, bb.x); x.y = fmaf(a, x.y, bb.y); x.z = fmaf(a, x.z, bb.z); x.w = fmaf(a, x.w, bb.w);
+            *reinterpret_cast<float4 *>(S + e) = x;
+        }
         __syncthreads();
         float acc[TR][TCc];
         if (worker) {
@@ -339,12 +343,8 @@ vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ C, const
 #pragma unroll
             for (int r = 0; r < TR; ++r) {
                 const size_t row = (size_t)(i0 + r) * DV + c0;
-                const float4 c0v = *reinterpret_cast<const float4 *>(C + fh * sdim + row);
-                const float4 c1v = *reinterpret_cast<const float4 *>(C + fh * sdim + row + 4);
-                const float4 n0 = make_float4(fmaf(a, acc[r][0], c0v.x), fmaf(a, acc[r][1], c0v.y),
-                                              fmaf(a, acc[r][2], c0v.z), fmaf(a, acc[r][3], c0v.w));
-                const float4 n1 = make_float4(fmaf(a, acc[r][4], c1v.x), fmaf(a, acc[r][5], c1v.y),
-                                              fmaf(a, acc[r][6], c1v.z), fmaf(a, acc[r][7], c1v.w));
+                const float4 n0 = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+                const float4 n1 = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
                 *reinterpret_cast<float4 *>(S + row) = n0;
                 *reinterpret_cast<float4 *>(S + row + 4) = n1;
                 if (!dir) {

@@ -216,6 +216,17 @@ namespace vda {
 // the chain's operand images (img_off), fetched by bulk copies.  Rows past
 // the frame's end are computed but not stored.
 // ---------------------------------------------------------------------------
+// Four consecutive outputs with one vector store (16 B fp32, 8 B bf16).
+__device__ __forceinline__ void store4(float *p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4 *>(p) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, float a, float b, float c, float d) {
+    uint2 v;
+    v.x = gdn::tc2::pack_bf16(a, b);
+    v.y = gdn::tc2::pack_bf16(c, d);
+    *reinterpret_cast<uint2 *>(p) = v;
+}
+
 template <int DV>
 struct ReadTcSmem {
     static constexpr int kQ = 0;                           // 2 key halves x [128 tok][64] bf16
@@ -317,7 +328,9 @@ vda_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const unsigned c
             tmem_wait_ld();
             if (u < U) {
 #pragma unroll
-                for (int q = 0; q < 16; ++q) dst[n0 + q] = from_f32<Tout>(hi[q] + lo[q]);
+                for (int q = 0; q < 16; q += 4)
+                    store4(dst + n0 + q, hi[q] + lo[q], hi[q + 1] + lo[q + 1], hi[q + 2] + lo[q + 2],
+                           hi[q + 3] + lo[q + 3]);
             }
         }
     } else if (tid == 0) {
