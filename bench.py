@@ -132,8 +132,8 @@ def kernel_algorithmic_bytes(name, w):
 # launch processes.  Keyed by (kernel, workload); absent means not captured
 # for this kernel as it stands.
 MEASURED_TRAFFIC_PER_TOKEN_HEAD = {
-    ("tc_fused", "stream480"): 319.89e6 / (12 * 8192),   # fused_kernel<128, 32, float>, T = 8192
-    ("tc_chain", "skewed"): 525.69e6 / (4 * 32 * 2048),  # chain_kernel<128, 64, float>, T = 2048
+    ("tc_fused", "stream480"): 327.29e6 / (12 * 8192),   # fused_kernel<128, 32, float>, T = 8192
+    ("tc_chain", "skewed"): 525.38e6 / (4 * 32 * 2048),  # chain_kernel<128, 64, float>, T = 2048
     ("tc_prep", "skewed"): 421.63e6 / (4 * 32 * 2048),   # prep_kernel<128>, T = 2048
 }
 
