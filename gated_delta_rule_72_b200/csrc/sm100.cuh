@@ -71,20 +71,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
     return false;
 }
 
-// Same, bounded by time: false once `limit_ns` of %globaltimer have passed.
-__device__ __forceinline__ unsigned long long global_ns_now() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ bool mbar_wait_ns(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_ns_now();
-    while (!mbar_try_wait(bar, parity))
-        if (global_ns_now() - t0 > limit_ns) return false;
-    return true;
-}
-
 // ---------------------------------------------------------------- TMA
 // 4-d tiled bulk tensor load global -> shared, completion counted on `bar`.
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar,
@@ -132,6 +118,15 @@ __device__ __forceinline__ unsigned long long global_ns() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+// Bounded wait on an mbarrier phase by time: false once `limit_ns` of
+// %globaltimer have passed without the phase completing.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > limit_ns) return false;
+    return true;
 }
 // Spin until *p >= v (acquire), for at most `limit_ns`; false on timeout.
 __device__ __forceinline__ bool spin_until_geq(const unsigned int *p, unsigned int v,

@@ -203,3 +203,44 @@ def test_readout_rejects_before_launch(lib):
     assert _readout(y=FAKE, y_dt=1) == -2
     # T = 0: nothing to do, no pointer needed
     assert _readout(T=0, o=None, z=None, y=None) == 0
+
+
+def _vda(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, alpha_frame=FAKE, beta=FAKE, state_in=None, state_in_bwd=None,
+             state_out=None, state_out_bwd=None, o=FAKE, B=1, F=3, U=40, H=2, dk=128, dv=128, bidir=1, dt=1,
+             o_dt=0, workspace=FAKE, ws_bytes=10, stream=None)
+    a.update(kw)
+    return _lib.gdn_vda_scan(*a.values())
+
+
+def test_vda_rejects_before_launch(lib):
+    """gdn_vda_scan argument checks (no CUDA call on these paths)."""
+    assert _vda(U=0) == -2
+    assert _vda(F=-1) == -2
+    assert _vda(dk=96) == -5
+    assert _vda(dt=7) == -3
+    assert _vda(q=None) == -1
+    assert _vda(k=FAKE + 8) == -4
+    assert _vda(state_in=FAKE + 4) == -4
+    assert _vda(state_out=FAKE + (1 << 20), state_out_bwd=FAKE + (1 << 20)) == -2   # both outputs in one buffer
+    assert _vda() == -6                                    # workspace too small
+    need = lib.gdn_vda_workspace_size(1, 3, 40, 2, 128, 128, 1)
+    # A and B per frame-head (64 KB each at d = 128), the two directions' states
+    assert need == 3 * 2 * (65536 + 65536) + 2 * 3 * 2 * 65536
+    assert lib.gdn_vda_workspace_size(1, 0, 40, 2, 128, 128, 1) == 0
+    assert lib.gdn_vda_workspace_size(1, 3, 0, 2, 128, 128, 1) == 0
+    # no frames: nothing to do, no pointer needed
+    assert _vda(F=0, q=None, k=None, v=None, alpha_frame=None, beta=None, o=None, workspace=None) == 0
+
+
+def test_python_api_refuses_cpu_tensors_for_new_calls():
+    import torch
+    import gated_delta_rule_72_b200 as gdn
+    q = torch.zeros(1, 6, 1, 64)
+    a = torch.ones(1, 6, 1)
+    with pytest.raises(ValueError):
+        gdn.vda_scan(q, q, q, torch.ones(1, 2, 1), a, 3)
+    with pytest.raises(ValueError):
+        gdn.vda_scan(q, q, q, torch.ones(1, 2, 1), a, 4)   # T = 6 is not a multiple of U = 4
+    with pytest.raises(ValueError):
+        gdn.readout_gate(q, q)
