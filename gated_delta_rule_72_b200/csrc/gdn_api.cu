@@ -644,7 +644,7 @@ gdn_status run_vda(const VdaArgs &a) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return GDN_ERR_CUDA;
         gdn::LaunchScope ls("vda_chain", a.stream);
-        kern<<<dim3(nbh, ndir), kChainThreads, smem, a.stream>>>(A, Bm, a.alpha_f, a.s_in, a.s_in_bwd, a.s_out,
+        kern<<<dim3(nbh, ndir, DV / kSlice), kChainThreads, smem, a.stream>>>(A, Bm, a.alpha_f, a.s_in, a.s_in_bwd, a.s_out,
                                                                 a.s_out_bwd, st, a.F, a.H);
         if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
     }

@@ -227,13 +227,16 @@ vda_factor_kernel(float *__restrict__ A)
 }
 
 // ---------------------------------------------------------------------------
-// The frame chain of one head and direction: S <- P_f (alpha_f S + B_f) per
-// frame, in the direction's order.  The state each readout needs goes to
-// `st` ([dir][F][B*H][DK][DV]): the causal direction stores S_f, the reverse
-// one R_{f+1} (before the frame is written).  Thread tile 4 rows x 8 columns
-// of S (DK x DV over 512 threads); P_f (symmetric: row k of P is column k) is
-// staged in shared memory.
+// The frame chain of one head, direction and slice of kSlice state columns
+// (the columns are independent: P_f acts on each alike): S <- P_f (alpha_f S
+// + B_f) per frame, in the direction's order.  The state each readout needs
+// goes to `st` ([dir][F][B*H][DK][DV]): the causal direction stores S_f, the
+// reverse one R_{f+1} (before the frame is written), as fp32 or (kImage) as
+// the tensor-core readout's operand image.  Thread tile 4 rows x 2 columns;
+// P_f (symmetric: row k of P is column k) is staged in shared memory.
 // ---------------------------------------------------------------------------
+constexpr int kSlice = 32;
+
 // State image for the tensor-core readout: [S_hi | S_lo] as bf16, the
 // operand layout of a 128B-swizzled MN-major B tile (rows = the key index,
 // groups of 64 columns 16 KB apart); S_hi + S_lo = S to about 2^-16.  Same
@@ -261,12 +264,10 @@ __device__ __forceinline__ void store_image_row8(unsigned char *img, int i, int 
 template <int DK, int DV>
 struct ChainSmem {
     static constexpr int kP = 0;                           // [DK][DK]
-    static constexpr int kS = kP + DK * DK * 4;            // [DK][DV]
-    static constexpr int kBytes = kS + DK * DV * 4;
+    static constexpr int kS = kP + DK * DK * 4;            // [DK][kSlice]
+    static constexpr int kBytes = kS + DK * kSlice * 4;
 };
 
-// kImage: the states for the readout are stored as tensor-core operand images
-// (store_image_row8) instead of fp32.
 template <int DK, int DV, bool kImage>
 __global__ void __launch_bounds__(kChainThreads)
 vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ Bm, const float *__restrict__ alpha_f,
@@ -274,22 +275,39 @@ vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ Bm, cons
                  float *__restrict__ st, int F, int H)
 {
     using SM = ChainSmem<DK, DV>;
-    constexpr int TR = 4, TCc = 8;
-    constexpr int NCT = DV / TCc;                      // column tiles
+    constexpr int TR = 4, TCc = 2;
+    constexpr int NCT = kSlice / TCc;                  // column tiles
     constexpr int kTiles = (DK / TR) * NCT;
-    static_assert(kTiles <= kChainThreads, "thread tiles");
+    static_assert(kTiles <= kChainThreads && DV % kSlice == 0, "thread tiles");
     extern __shared__ __align__(16) unsigned char csm[];
     float *Ps = reinterpret_cast<float *>(csm + SM::kP);
     float *S = reinterpret_cast<float *>(csm + SM::kS);
-    const int bh = blockIdx.x, nbh = gridDim.x, dir = blockIdx.y;
+    const int bh = blockIdx.x, nbh = gridDim.x, dir = blockIdx.y, j0 = blockIdx.z * kSlice;
     const int b = bh / H, h = bh % H;
     const int tid = threadIdx.x;
     const float *src0 = dir ? s_in_bwd : s_in;   // (an output state may be its own input)
     float *dst_end = dir ? s_out_bwd : s_out;
     const size_t sdim = (size_t)DK * DV;
-    for (int e = tid; e < DK * DV; e += kChainThreads) S[e] = src0 ? src0[bh * sdim + e] : 0.f;
+    for (int e = tid; e < DK * kSlice; e += kChainThreads) {
+        const int i = e / kSlice, c = e % kSlice;
+        S[e] = src0 ? src0[bh * sdim + (size_t)i * DV + j0 + c] : 0.f;
+    }
     const bool worker = tid < kTiles;
     const int i0 = (tid / NCT) * TR, c0 = (tid % NCT) * TCc;
+    // the slice's state to `dst` (fp32, or operand image: 8 columns per 16-byte chunk)
+    auto store_state = [&](float *dst) {
+        if (kImage) {
+            for (int e = tid; e < DK * (kSlice / 8); e += kChainThreads) {
+                const int i = e / (kSlice / 8), q = e % (kSlice / 8);
+                store_image_row8<DV>(reinterpret_cast<unsigned char *>(dst), i, j0 + 8 * q, S + i * kSlice + 8 * q);
+            }
+        } else {
+            for (int e = tid; e < DK * kSlice; e += kChainThreads) {
+                const int i = e / kSlice, c = e % kSlice;
+                dst[(size_t)i * DV + j0 + c] = S[e];
+            }
+        }
+    };
 
     for (int step = 0; step < F; ++step) {
         const int f = dir ? F - 1 - step : step;
@@ -297,26 +315,13 @@ vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ Bm, cons
         const float a = alpha_f[((size_t)b * F + f) * H + h];
         float *dst = st + ((size_t)dir * F * nbh + fh) * sdim;
         __syncthreads();                                   // S complete, P free
-        if (dir) {   // the reverse readout of frame f reads R_{f+1}
-            if (kImage) {
-                if (worker)
-#pragma unroll
-                    for (int r = 0; r < TR; ++r)
-                        store_image_row8<DV>(reinterpret_cast<unsigned char *>(dst), i0 + r, c0,
-                                             S + (i0 + r) * DV + c0);
-            } else {
-                for (int e = tid * 4; e < DK * DV; e += kChainThreads * 4)
-                    *reinterpret_cast<float4 *>(dst + e) = *reinterpret_cast<const float4 *>(S + e);
-            }
-        }
+        if (dir) store_state(dst);                         // the reverse readout of frame f reads R_{f+1}
         for (int e = tid * 4; e < DK * DK; e += kChainThreads * 4)
             *reinterpret_cast<float4 *>(Ps + e) = *reinterpret_cast<const float4 *>(P + fh * DK * DK + e);
-        __syncthreads();   // (the reverse direction's store above has read S)
-        for (int e = tid * 4; e < DK * DV; e += kChainThreads * 4) {   // S <- alpha S + B
-            float4 x = *reinterpret_cast<const float4 *>(S + e);
-            const float4 bb = *reinterpret_cast<const float4 *>(Bm + fh * sdim + e);
-            x.x = fmaf(a, x.x, bb.x); x.y = fmaf(a, x.y, bb.y); x.z = fmaf(a, x.z, bb.z); x.w = fmaf(a, x.w, bb.w);
-            *reinterpret_cast<float4 *>(S + e) = x;
+        __syncthreads();
+        for (int e = tid; e < DK * kSlice; e += kChainThreads) {   // S <- alpha S + B
+            const int i = e / kSlice, c = e % kSlice;
+            S[e] = fmaf(a, S[e], Bm[fh * sdim + (size_t)i * DV + j0 + c]);
         }
         __syncthreads();
         float acc[TR][TCc];
@@ -325,43 +330,34 @@ vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ Bm, cons
             for (int r = 0; r < TR; ++r)
 #pragma unroll
                 for (int cc = 0; cc < TCc; ++cc) acc[r][cc] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
             for (int kk = 0; kk < DK; ++kk) {
                 const float4 pv = *reinterpret_cast<const float4 *>(Ps + kk * DK + i0);   // P[i0..][kk]
+                const float2 sv = *reinterpret_cast<const float2 *>(S + kk * kSlice + c0);
                 const float pa[TR] = {pv.x, pv.y, pv.z, pv.w};
-                const float4 s0 = *reinterpret_cast<const float4 *>(S + kk * DV + c0);
-                const float4 s1 = *reinterpret_cast<const float4 *>(S + kk * DV + c0 + 4);
-                const float sv[TCc] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-                for (int r = 0; r < TR; ++r)
-#pragma unroll
-                    for (int cc = 0; cc < TCc; ++cc) acc[r][cc] = fmaf(pa[r], sv[cc], acc[r][cc]);
+                for (int r = 0; r < TR; ++r) {
+                    acc[r][0] = fmaf(pa[r], sv.x, acc[r][0]);
+                    acc[r][1] = fmaf(pa[r], sv.y, acc[r][1]);
+                }
             }
         }
         __syncthreads();                                   // every read of the old S is done
-        if (worker) {
+        if (worker)
 #pragma unroll
-            for (int r = 0; r < TR; ++r) {
-                const size_t row = (size_t)(i0 + r) * DV + c0;
-                const float4 n0 = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-                const float4 n1 = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
-                *reinterpret_cast<float4 *>(S + row) = n0;
-                *reinterpret_cast<float4 *>(S + row + 4) = n1;
-                if (!dir) {
-                    if (kImage) {
-                        const float x8[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
-                        store_image_row8<DV>(reinterpret_cast<unsigned char *>(dst), i0 + r, c0, x8);
-                    } else {
-                        *reinterpret_cast<float4 *>(dst + row) = n0;
-                        *reinterpret_cast<float4 *>(dst + row + 4) = n1;
-                    }
-                }
-            }
+            for (int r = 0; r < TR; ++r)
+                *reinterpret_cast<float2 *>(S + (i0 + r) * kSlice + c0) = make_float2(acc[r][0], acc[r][1]);
+        if (!dir) {
+            __syncthreads();
+            store_state(dst);
         }
     }
     __syncthreads();
     if (dst_end)
-        for (int e = tid; e < DK * DV; e += kChainThreads) dst_end[bh * sdim + e] = S[e];
+        for (int e = tid; e < DK * kSlice; e += kChainThreads) {
+            const int i = e / kSlice, c = e % kSlice;
+            dst_end[bh * sdim + (size_t)i * DV + j0 + c] = S[e];
+        }
 }
 
 // ---------------------------------------------------------------------------
