@@ -65,7 +65,7 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------
-# algorithmic traffic and work (per token-head), see the design doc section 6
+# algorithmic traffic and work (per token-head)
 # ---------------------------------------------------------------------------
 def bytes_per_token_head(w, out_bytes=4):
     ib = 4 if w.dtype == "f32" else 2
