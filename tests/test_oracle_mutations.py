@@ -92,3 +92,53 @@ def test_planted_mistake_is_caught(mutation, tmp_path):
     finally:
         oracle._lib = real
     assert failed, "no pin caught the planted mistake %r" % mutation
+
+
+# --------------------------------------------------------------------------
+# The numpy oracles (frame-wise operator, readout epilogue): a mutated copy of
+# the function's source replaces it while the pins run.
+# --------------------------------------------------------------------------
+NUMPY_MUTATIONS = {
+    # frame-wise operator
+    "vda_beta_dropped_in_gram": ("vda_scan", "K.T @ (be[:, None] * K)", "K.T @ K"),
+    "vda_beta_dropped_in_write": ("vda_scan", "K.T @ (be[:, None] * V)", "K.T @ V"),
+    "vda_plain_additive_write": ("vda_scan", "S = np.linalg.solve(eye + A, alpha_f[b, f, h] * S + Bm)",
+                                 "S = alpha_f[b, f, h] * (S - A @ S) + Bm"),
+    "vda_decay_after_solve": ("vda_scan", "S = np.linalg.solve(eye + A, alpha_f[b, f, h] * S + Bm)",
+                              "S = alpha_f[b, f, h] * np.linalg.solve(eye + A, S) + Bm"),
+    "vda_readout_before_write": ("vda_scan", """                    S = np.linalg.solve(eye + A, alpha_f[b, f, h] * S + Bm)
+                    o[b, t, h] += q[b, t, h] @ S""", """                    o[b, t, h] += q[b, t, h] @ S
+                    S = np.linalg.solve(eye + A, alpha_f[b, f, h] * S + Bm)"""),
+    "vda_reverse_not_strict": ("vda_scan", """                    o[b, t, h] += q[b, t, h] @ R
+                    R = np.linalg.solve(eye + A, alpha_f[b, f, h] * R + Bm)""", """                    R = np.linalg.solve(eye + A, alpha_f[b, f, h] * R + Bm)
+                    o[b, t, h] += q[b, t, h] @ R"""),
+    "vda_state_in_ignored": ("vda_scan", "S = np.zeros((dk, dv)) if s0 is None else s0[b, h].copy()",
+                             "S = np.zeros((dk, dv))"),
+    # readout epilogue
+    "readout_no_norm": ("readout_gate", "inv = 1.0 / np.sqrt(np.mean(row * row) + eps)", "inv = 1.0"),
+    "readout_sum_not_mean": ("readout_gate", "np.mean(row * row)", "np.sum(row * row)"),
+    "readout_gate_inverted": ("readout_gate", "(1.0 + np.exp(-flat_z[r, j]))", "(1.0 + np.exp(flat_z[r, j]))"),
+    "readout_gain_dropped": ("readout_gate", "row[j] * inv * g[j]", "row[j] * inv"),
+    "readout_eps_outside": ("readout_gate", "np.sqrt(np.mean(row * row) + eps)", "(np.sqrt(np.mean(row * row)) + eps)"),
+}
+
+
+@pytest.mark.parametrize("mutation", sorted(NUMPY_MUTATIONS))
+def test_planted_mistake_in_numpy_oracle_is_caught(mutation):
+    fname, old, new = NUMPY_MUTATIONS[mutation]
+    real = getattr(oracle, fname)
+    src = inspect.getsource(real)
+    assert src.count(old) >= 1, "mutation anchor not found: %s" % mutation
+    ns = {}
+    exec(compile(src.replace(old, new), "<mutated %s>" % fname, "exec"), oracle.__dict__, ns)
+    failed = []
+    setattr(oracle, fname, ns[fname])
+    try:
+        for name, fn in _pin_functions():
+            try:
+                fn()
+            except AssertionError:
+                failed.append(name)
+    finally:
+        setattr(oracle, fname, real)
+    assert failed, "no pin caught the planted mistake %r" % mutation
