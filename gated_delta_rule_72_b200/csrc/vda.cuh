@@ -1,4 +1,6 @@
-// vda.cuh -- frame-wise delta operator (VDA) on the CUDA cores, fp32.
+// vda.cuh -- frame-wise delta operator (VDA): the kernels that run on the
+// CUDA cores, in fp32 (vda_tc.cuh has the tensor-core Gram and readout used
+// for bf16 inputs with d_k = 128).
 //
 // The sequence is split into F frames of U consecutive tokens.  For frame f
 // (keys K_f: U x dk, values V_f: U x dv, per-token write strengths beta, a
@@ -11,13 +13,13 @@
 // f: o_u = S_f^T q_u (+ R_{f+1}^T q_u for a bidirectional scan: the frames
 // after f only).
 //
-// Four kernels:
+// Four steps:
 //   vda_gram    (frame x head, fully parallel)  A_f and B_f
 //   vda_factor  (frame x head, fully parallel)  P_f = (I + A_f)^{-1} by a
 //               Cholesky factorisation: none of it depends on the state
-//   vda_chain   (head x direction, sequential over frames)  S <- P_f (alpha_f S
-//               + B_f), the state in shared memory; stores the state each
-//               frame's readout uses
+//   vda_chain   (head x direction x 32 state columns, sequential over frames)
+//               S <- P_f (alpha_f S + B_f), the slice of the state in shared
+//               memory; stores the state each frame's readout uses
 //   vda_readout (token block x head, fully parallel)  o = Q (S + R)
 #pragma once
 
