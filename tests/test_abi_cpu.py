@@ -244,3 +244,22 @@ def test_python_api_refuses_cpu_tensors_for_new_calls():
         gdn.vda_scan(q, q, q, torch.ones(1, 2, 1), a, 4)   # T = 6 is not a multiple of U = 4
     with pytest.raises(ValueError):
         gdn.readout_gate(q, q)
+
+
+def _declared_arity():
+    """Parameter count of every GDN_API function in the header."""
+    text = open(HEADER).read()
+    out = {}
+    for m in re.finditer(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    """The ctypes binding passes exactly as many arguments as each C function
+    declares (a missing or extra argument would shift every later one)."""
+    arity = _declared_arity()
+    assert set(arity) == set(_lib.SIGNATURES), set(arity) ^ set(_lib.SIGNATURES)
+    for name, (_, argtypes) in _lib.SIGNATURES.items():
+        assert len(argtypes) == arity[name], (name, len(argtypes), arity[name])
