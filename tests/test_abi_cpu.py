@@ -263,3 +263,24 @@ def test_binding_signatures_match_the_header():
     assert set(arity) == set(_lib.SIGNATURES), set(arity) ^ set(_lib.SIGNATURES)
     for name, (_, argtypes) in _lib.SIGNATURES.items():
         assert len(argtypes) == arity[name], (name, len(argtypes), arity[name])
+
+
+def test_binding_argument_types_match_the_header():
+    """Each argument's ctypes type fits its C type: pointers as pointers,
+    int and enum as c_int, size_t as c_size_t, float as c_float."""
+    text = open(HEADER).read()
+    for m in re.finditer(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(([^)]*)\)\s*;", text):
+        name, params = m.group(1), m.group(2).strip()
+        if params in ("", "void"):
+            continue
+        argtypes = _lib.SIGNATURES[name][1]
+        for decl, ct in zip([p.strip() for p in params.split(",")], argtypes):
+            if "*" in decl:
+                assert ct is ctypes.c_void_p or issubclass(ct, (ctypes._Pointer, ctypes.c_char_p)), (name, decl, ct)
+            elif decl.startswith("size_t"):
+                assert ct is ctypes.c_size_t, (name, decl, ct)
+            elif decl.startswith("float"):
+                assert ct is ctypes.c_float, (name, decl, ct)
+            else:
+                assert decl.split()[0] in ("int", "gdn_dtype", "gdn_status"), (name, decl)
+                assert ct is ctypes.c_int, (name, decl, ct)
