@@ -5,11 +5,13 @@
                     [--impl ours|reference]
 
 A step is one pass of the whole scan over one batch of synthetic inputs that
-are already resident in HBM: for the default workload, stream480
-(B=1, H=12, T=32,760, d_k=d_v=128, bf16 q/k/v, fp32 gates, fp32 output and
-state), one gdn_scan_causal call.  Its inputs (~500 MB) are larger than the
-126 MB L2, so no flush is needed between steps; for workloads smaller than
-L2 a 256 MB buffer is written between timed steps, outside the events.
+are already resident in HBM: for the default workload, skewed (B=4, H=32,
+T=16,384, d_k=d_v=128, bf16 q/k/v, fp32 gates, fp32 output and state; the
+largest single-call workload), one gdn_scan_causal call.  Its inputs
+(~1.6 GB) are larger than the 126 MB L2, so no flush is needed between steps;
+for workloads smaller than L2 a 256 MB buffer is written between timed steps,
+outside the events.  After the headline workload the other bf16 workloads
+(--others) are timed the same way and reported under `others`.
 
 Metric: Mtokens/s = B*H*T per step / step time.  Time is measured with CUDA
 events on the launching stream after W warm-up steps, bracketed by a barrier
@@ -25,7 +27,9 @@ API with the inputs copied from pinned host memory and the output and state
 read back inside the timed region), `clocks` (nvidia-smi samples taken during
 the timed region), `gpu_launches` (kernels the library launched in the
 timed region, from its own launch counter) and, for the rollout workload,
-`graph` (the same step captured once in a CUDA graph and replayed).
+`graph` (the same step captured once in a CUDA graph and replayed),
+`device_timeouts` (bounded device-side waits that gave up during the run,
+read from the library; a non-zero count marks the line invalid).
 
 `--impl reference` times the FP64 oracle (the reference implementation of
 this build) on the host cores instead: each step is a bounded sample of the
@@ -103,8 +107,8 @@ def vda_kernel_flops(w):
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def algorithmic_bytes_per_step(w):
-    b = w.token_heads * bytes_per_token_head(w)
+def algorithmic_bytes_per_step(w, out_bytes=4):
+    b = w.token_heads * bytes_per_token_head(w, out_bytes)
     if w.mode == "rollout":
         b += w.calls * 2 * state_bytes_per_call(w)       # state read + written per call
     elif w.mode == "causal":
@@ -114,11 +118,11 @@ def algorithmic_bytes_per_step(w):
 
 # Per kernel: which algorithmic bytes (per token-head) it moves.  The prep
 # kernel reads q, k, v and the gates; the chain kernel writes o (and the
-# state).  A fused kernel moves all of them.
-def kernel_algorithmic_bytes(name, w):
+# state).  A fused kernel moves all of them.  out_bytes: element size of o.
+def kernel_algorithmic_bytes(name, w, out_bytes=4):
     ib = 4 if w.dtype == "f32" else 2
     reads = ib * (2 * w.dk + w.dv) + 8
-    writes = 4 * w.dv
+    writes = out_bytes * w.dv
     if "prep" in name:
         return reads
     if "chain" in name:
@@ -132,9 +136,6 @@ def kernel_algorithmic_bytes(name, w):
 # launch processes.  Keyed by (kernel, workload); absent means not captured
 # for this kernel as it stands.
 MEASURED_TRAFFIC_PER_TOKEN_HEAD = {
-    ("tc_fused", "stream480"): 327.29e6 / (12 * 8192),   # fused_kernel<128, 32, float>, T = 8192
-    ("tc_chain", "skewed"): 525.38e6 / (4 * 32 * 2048),  # chain_kernel<128, 64, float>, T = 2048
-    ("tc_prep", "skewed"): 421.63e6 / (4 * 32 * 2048),   # prep_kernel<128>, T = 2048
 }
 
 
@@ -365,13 +366,132 @@ def oracle_sample(w, target_s):
     return units / ts / 1e6, threads, desc, Ts
 
 
+def device_timeouts(gdn):
+    """Bounded device-side waits of the library that gave up so far (the
+    library's own counter; a timed result is valid only while it stays 0)."""
+    try:
+        return int(gdn.gdn_device_timeouts())
+    except Exception:   # noqa: BLE001  (reported as unknown, never as zero)
+        return -1
+
+
+def roofline_of(w, ktimes, steps, units, peaks, peak_src):
+    """The dominant kernel's achieved rate against its roofline, from the
+    per-kernel CUDA-event times of the timed region."""
+    if not ktimes:
+        return None
+    name, (tot_ms, n) = max(ktimes.items(), key=lambda kv: kv[1][0])
+    per_launch_ms = tot_ms / n
+    launches_per_step = n / steps
+    units_per_launch = units / launches_per_step
+    bound = "tensor" if w.mode == "bidir" and "chain" not in name else "hbm"
+    if w.mode == "vda":
+        bound = "alu"     # fp32 on the CUDA cores
+    extra = {}
+    if bound == "alu":
+        alg = vda_kernel_flops(w).get(name, 0.0) * units_per_launch
+        achieved = alg / (per_launch_ms * 1e-3) / 1e12
+        peak = FP32_ALU_TFLOPS
+        unit = "TFLOP/s"
+    elif bound == "hbm":
+        alg = kernel_algorithmic_bytes(name, w) * units_per_launch
+        achieved = alg / (per_launch_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+        # the same kernel against the survey's byte count, o in bf16
+        alg16 = kernel_algorithmic_bytes(name, w, out_bytes=2) * units_per_launch
+        extra = {"frac_bf16_out_bytes": alg16 / (per_launch_ms * 1e-3) / 1e9 / peak,
+                 "bytes_per_token_head": kernel_algorithmic_bytes(name, w),
+                 "bytes_per_token_head_bf16_out": kernel_algorithmic_bytes(name, w, out_bytes=2)}
+    else:
+        alg = flops_per_token_head(w) * units_per_launch
+        achieved = alg / (per_launch_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+    total_ms = sum(t for t, _ in ktimes.values())
+    tph = MEASURED_TRAFFIC_PER_TOKEN_HEAD.get((name, w.name))
+    traffic = tph * units_per_launch if tph is not None else None
+    roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": traffic, "kernel": name,
+            "peak_source": ("derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1.965 GHz" if bound == "alu" else
+                            "%s (%s)" % (peak_src, "MEASURED_PEAKS.json" if peak_src == "measured"
+                                         else "pool fallback")),
+            "kernel_ms_per_launch": per_launch_ms,
+            "kernel_share": tot_ms / total_ms if total_ms else None,
+            "kernels": {k: {"ms_per_step": t / steps, "launches_per_step": c / steps}
+                        for k, (t, c) in ktimes.items()}}
+    roof.update(extra)
+    return roof
+
+
+def step_roofline(w, ms, peaks):
+    """The whole step against its roofline: bytes at HBM bandwidth vs FLOPs at
+    the tensor peak; bytes with o in fp32 (as written here) and in bf16 (the
+    survey's count)."""
+    t_flop = w.token_heads * flops_per_token_head(w) / (peaks["bf16_tflops"] * 1e12)
+    out = {}
+    for key, ob in (("", 4), ("_bf16_out", 2)):
+        t_mem = algorithmic_bytes_per_step(w, ob) / (peaks["hbm_gbs"] * 1e9)
+        t = max(t_mem, t_flop)
+        out["t_roofline_ms" + key] = t * 1e3
+        out["bound" + key] = "hbm" if t_mem >= t_flop else "tensor"
+        out["frac" + key] = t / (ms * 1e-3)
+    return out
+
+
+def measure(torch, gdn, w, device, args, dist, rank, clocks=True):
+    """Warm up, then time args.steps steps of workload w with per-kernel
+    events on; the clocks are sampled during the timed region."""
+    step = GPUStep(w, device)
+    for _ in range(max(3, args.warmup)):
+        step.between()
+        step.run()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(range(args.gpus)) if clocks else None
+    if sampler:
+        # nvidia-smi takes a moment to start sampling: keep the GPU busy with
+        # extra untimed steps for ~1 s so samples cover the load up to the
+        # timed region, which follows immediately
+        sampler.start()
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
+            step.run()
+            torch.cuda.synchronize()
+    gdn.gdn_read_kernel_timing()                  # drop anything recorded so far
+    n0 = gdn.gdn_launch_count()
+    gdn.gdn_set_kernel_timing(1)
+    ms = timed(torch, step.run, step.between, args.steps, dist)
+    gdn.gdn_set_kernel_timing(0)
+    launches = gdn.gdn_launch_count() - n0
+    clk = sampler.stop() if sampler else None
+    ktimes = gdn.gdn_read_kernel_timing()
+    ms = max_over_ranks(torch, dist, ms, device)
+    units = w.token_heads                          # per GPU per step
+    peaks, peak_src = load_peaks()
+    return {"step": step, "ms": ms, "value": whole_job_value(args.gpus, units, ms),
+            "roof": roofline_of(w, ktimes, args.steps, units, peaks, peak_src),
+            "step_roof": step_roofline(w, ms, peaks), "clocks": clk, "launches": launches}
+
+
+def workload_config(w, gpus):
+    return {"workload": "%s (%s B=%d H=%d T=%d%s d_k=%d d_v=%d, %s in, fp32 out/state, %s gates)"
+            % (w.name, w.mode, w.B, w.H, w.T, (" x %d calls" % w.calls) if w.calls > 1 else "",
+               w.dk, w.dv, w.dtype, w.gates),
+            "B": w.B, "H": w.H, "T": w.total_T, "d_k": w.dk, "d_v": w.dv,
+            **({"frame": w.frame} if w.mode == "vda" else {"chunk": 64}),
+            "parallelism": "replicas%d (independent (b,h) problems per GPU)" % gpus}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="stream480",
+    ap.add_argument("--workload", default="skewed",
                     choices=["stream480", "bidir720", "rollout", "skewed", "tiny", "vda480"])
+    ap.add_argument("--others", default="stream480,bidir720,rollout",
+                    help="comma-separated workloads timed after the headline one (device time only); "
+                         "empty: none")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target length of the oracle CPU-baseline sample")
@@ -389,12 +509,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    config = {"workload": "%s (%s B=%d H=%d T=%d%s d_k=%d d_v=%d, %s in, fp32 out/state, %s gates)"
-              % (w.name, w.mode, w.B, w.H, w.T, (" x %d calls" % w.calls) if w.calls > 1 else "",
-                 w.dk, w.dv, w.dtype, w.gates),
-              "B": w.B, "H": w.H, "T": w.total_T, "d_k": w.dk, "d_v": w.dv,
-              **({"frame": w.frame} if w.mode == "vda" else {"chunk": 64}),
-              "parallelism": "replicas%d (independent (b,h) problems per GPU)" % args.gpus}
+    config = workload_config(w, args.gpus)
 
     if args.impl == "reference":
         if rank != 0:
@@ -440,81 +555,13 @@ def main():
     torch.cuda.set_device(device)
     gdn.load()
 
-    step = GPUStep(w, device)
-    for _ in range(max(3, args.warmup)):
-        step.between()
-        step.run()
-    torch.cuda.synchronize()
-
-    # ---- the timed region: K steps, per-kernel events on, clocks sampled
-    sampler = ClockSampler(range(args.gpus)) if rank == 0 else None
-    if sampler:
-        # nvidia-smi takes a moment to start sampling: keep the GPU busy with
-        # extra untimed steps for ~1 s so samples cover the load up to the
-        # timed region, which follows immediately
-        sampler.start()
-        t_end = time.time() + 1.0
-        while time.time() < t_end:
-            step.run()
-            torch.cuda.synchronize()
-    gdn.gdn_read_kernel_timing()                  # drop anything recorded so far
-    n0 = gdn.gdn_launch_count()
-    gdn.gdn_set_kernel_timing(1)
-    ms = timed(torch, step.run, step.between, args.steps, dist)
-    gdn.gdn_set_kernel_timing(0)
-    launches = gdn.gdn_launch_count() - n0
-    clocks = sampler.stop() if sampler else None
-    ktimes = gdn.gdn_read_kernel_timing()
-    ms = max_over_ranks(torch, dist, ms, device)
-
-    units = w.token_heads                          # per GPU per step
-    value = whole_job_value(args.gpus, units, ms)
-
-    # ---- roofline of the dominant kernel
-    peaks, peak_src = load_peaks()
-    dom = max(ktimes.items(), key=lambda kv: kv[1][0]) if ktimes else None
-    roof = None
-    if dom:
-        name, (tot_ms, n) = dom
-        per_launch_ms = tot_ms / n
-        launches_per_step = n / args.steps
-        units_per_launch = units / launches_per_step
-        bound = "tensor" if w.mode == "bidir" and "chain" not in name else "hbm"
-        if w.mode == "vda":
-            bound = "alu"     # fp32 on the CUDA cores
-        if bound == "alu":
-            alg = vda_kernel_flops(w).get(name, 0.0) * units_per_launch
-            achieved = alg / (per_launch_ms * 1e-3) / 1e12
-            peak = FP32_ALU_TFLOPS
-            unit = "TFLOP/s"
-        elif bound == "hbm":
-            alg = kernel_algorithmic_bytes(name, w) * units_per_launch
-            achieved = alg / (per_launch_ms * 1e-3) / 1e9
-            peak = peaks["hbm_gbs"]
-            unit = "GB/s"
-        else:
-            alg = flops_per_token_head(w) * units_per_launch
-            achieved = alg / (per_launch_ms * 1e-3) / 1e12
-            peak = peaks["bf16_tflops"]
-            unit = "TFLOP/s"
-        total_ms = sum(t for t, _ in ktimes.values())
-        tph = MEASURED_TRAFFIC_PER_TOKEN_HEAD.get((name, w.name))
-        traffic = tph * units_per_launch if tph is not None else None
-        roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": traffic, "kernel": name,
-                "peak_source": ("derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1.965 GHz" if bound == "alu" else
-                                "%s (%s)" % (peak_src, "MEASURED_PEAKS.json" if peak_src == "measured"
-                                             else "pool fallback")),
-                "kernel_ms_per_launch": per_launch_ms,
-                "kernel_share": tot_ms / total_ms if total_ms else None,
-                "kernels": {k: {"ms_per_step": t / args.steps, "launches_per_step": c / args.steps}
-                            for k, (t, c) in ktimes.items()}}
-    # whole step against its roofline (bytes at HBM bandwidth vs FLOPs at tensor peak)
-    t_mem = algorithmic_bytes_per_step(w) / (peaks["hbm_gbs"] * 1e9)
-    t_flop = w.token_heads * flops_per_token_head(w) / (peaks["bf16_tflops"] * 1e12)
-    step_roof = {"t_roofline_ms": max(t_mem, t_flop) * 1e3,
-                 "bound": "hbm" if t_mem >= t_flop else "tensor",
-                 "frac": max(t_mem, t_flop) / (ms * 1e-3)}
+    timeouts0 = device_timeouts(gdn)
+    m = measure(torch, gdn, w, device, args, dist, rank, clocks=(rank == 0))
+    step, ms, value, roof, step_roof, clocks, launches = (m[k] for k in (
+        "step", "ms", "value", "roof", "step_roof", "clocks", "launches"))
+    units = w.token_heads
+    l2_note = ("inputs larger than L2, no flush" if step.flush is None
+               else "L2 flushed between steps (256 MB write)")
 
     # ---- the streaming rollout replayed from a CUDA graph (device-timed like value)
     graph = None
@@ -534,17 +581,42 @@ def main():
         rate, threads, desc, _ = oracle_sample(w, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
 
+    # ---- the other workloads, device time only (every rank, same order)
+    others = {}
+    del step, m
+    torch.cuda.empty_cache()
+    for name in [x for x in args.others.split(",") if x and x != w.name]:
+        wo = inputs.WORKLOADS[name]
+        mo = measure(torch, gdn, wo, device, args, dist, rank, clocks=(rank == 0))
+        rec = {"value": mo["value"], "unit": UNIT, "ms_per_step": mo["ms"],
+               "config": workload_config(wo, args.gpus), "roofline": mo["roof"],
+               "step_roofline": mo["step_roof"], "clocks": mo["clocks"], "gpu_launches": mo["launches"]}
+        if wo.mode == "rollout":
+            gms = max_over_ranks(torch, dist, graph_replay_ms(torch, mo["step"], args.steps, dist), device)
+            rec["graph"] = {"value": whole_job_value(args.gpus, wo.token_heads, gms), "unit": UNIT,
+                            "ms_per_step": gms, "calls_per_step": wo.calls}
+        others[name] = rec
+        del mo
+        torch.cuda.empty_cache()
+    timeouts1 = device_timeouts(gdn)
+    n_timeouts = timeouts1 - timeouts0 if min(timeouts0, timeouts1) >= 0 else None
+
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": dict(config, l2=("inputs larger than L2, no flush" if step.flush is None
-                                           else "L2 flushed between steps (256 MB write)")),
+                "config": dict(config, l2=l2_note),
                 "roofline": roof, "step_roofline": step_roof,
                 "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches}
         if graph is not None:
             line["graph"] = graph
+        if others:
+            line["others"] = others
+        line["device_timeouts"] = n_timeouts
+        if n_timeouts != 0:
+            line["valid"] = False
+            line["note"] = "a bounded device-side wait gave up (or the count is unknown): not a result"
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

@@ -8,5 +8,5 @@ not on a CUDA device.
 """
 from ._lib import GDNError, gdn_scan_bidir, gdn_scan_bidir_states, gdn_scan_causal, gdn_status_string, gdn_step, \
     gdn_version, gdn_workspace_size, gdn_launch_count, gdn_set_kernel_timing, \
-    gdn_read_kernel_timing, gdn_device_timeouts, gdn_set_short_call_tokens, gdn_readout_gate, gdn_vda_scan, gdn_vda_workspace_size, load  # noqa: F401
+    gdn_read_kernel_timing, gdn_device_timeouts, gdn_set_short_call_tokens, gdn_set_chain_segments, gdn_readout_gate, gdn_vda_scan, gdn_vda_workspace_size, load  # noqa: F401
 from .api import readout_gate, scan_bidir, scan_causal, step, vda_scan, workspace_size  # noqa: F401

@@ -38,6 +38,7 @@ SIGNATURES = {
     "gdn_device_timeouts": (_I, [ctypes.POINTER(ctypes.c_uint)]),
     "gdn_set_kernel_timing": (None, [_I]),
     "gdn_set_short_call_tokens": (_I, [_I]),
+    "gdn_set_chain_segments": (_I, [_I]),
     "gdn_read_kernel_timing": (_I, [ctypes.c_char_p, _I, ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(_I), _I]),
 }
@@ -149,6 +150,13 @@ def gdn_set_short_call_tokens(max_t):
     max_t < 0 restores the automatic choice.  Returns the previous setting
     (-1 for automatic)."""
     return int(load().gdn_set_short_call_tokens(int(max_t)))
+
+
+def gdn_set_chain_segments(g):
+    """Segments per chunk walk of the tensor-core path (sequence
+    parallelism); g < 1 restores the automatic choice.  Returns the previous
+    setting (-1 for automatic)."""
+    return int(load().gdn_set_chain_segments(int(g)))
 
 
 def gdn_read_kernel_timing(max_kernels=16, name_len=64):

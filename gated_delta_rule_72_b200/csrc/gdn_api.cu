@@ -197,27 +197,29 @@ bool use_tc(gdn_dtype dt, int dk, int dv) {
 }
 
 size_t tc_record_bytes(int dv) {
-    return dv == 128 ? gdn::tc2::Rec<128>::kBytes : gdn::tc2::Rec<64>::kBytes;
+    return dv == 128 ? gdn::tc2::Rec<128>::kStride : gdn::tc2::Rec<64>::kStride;
 }
 
-// Tensor-core path workspace: one record per chunk, head and direction; then,
-// bidirectional only, the fp32 output piece buffers of the two directions
-// (the causal one is o itself when o is fp32) and one counter per piece.
-size_t tc_pair_counters(int B, int T, int H, int dv) {
+// Tensor-core path workspace: one record per chunk, head and direction, one
+// ready flag and one log bound per record; then, bidirectional only, the fp32
+// sum buffer of the two directions (bf16 o; an fp32 o is its own sum) and one
+// counter per output tile.
+size_t tc_pair_counters(int B, int T, int H) {
     const size_t nC = (size_t)(T + kChunk - 1) / kChunk;
-    return (size_t)B * H * nC * (dv / 32);   // one per output tile of the narrowest slices
+    return (size_t)B * H * nC;   // one per (b, h, chunk) output tile
 }
 
 size_t plan_workspace(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt, int bidir) {
     if (T == 0) return 0;
     if (use_tc(dt, dk, dv)) {
         const size_t nC = (size_t)(T + kChunk - 1) / kChunk;
-        size_t bytes = round_up((bidir ? 2 : 1) * (size_t)B * H * nC * tc_record_bytes(dv), 256);
-        bytes += round_up((bidir ? 2 : 1) * (size_t)B * H * nC * sizeof(unsigned int), 256);   // ready flags
+        const size_t nrec = (bidir ? 2 : 1) * (size_t)B * H * nC;
+        size_t bytes = round_up(nrec * tc_record_bytes(dv), 256);
+        bytes += round_up(nrec * sizeof(unsigned int), 256);   // ready flags
+        bytes += round_up(nrec * sizeof(float), 256);          // log bounds of the chunk maps
         if (bidir) {
-            // the two directions add up in fp32: in o itself, or (bf16 o) in a buffer
             if (o_dt == GDN_BF16) bytes += round_up((size_t)B * T * H * dv * sizeof(float), 256);
-            bytes += round_up(tc_pair_counters(B, T, H, dv) * sizeof(unsigned int), 256);
+            bytes += round_up(tc_pair_counters(B, T, H) * sizeof(unsigned int), 256);
         }
         return bytes;
     }
@@ -283,9 +285,68 @@ int sm_count() {
     return n;
 }
 
+// Output tile map: fp32 boxes of 32 columns, bf16 boxes of 64 (128-byte rows,
+// 128B swizzle, as the chain stages them).
+bool encode_out_map(CUtensorMap *m, const void *target, const Args &a, int dv, bool f32) {
+    return encode_map(m, target, a.B, a.T, a.H, dv, f32 ? 32 : 64, 128, f32 ? 4 : 2);
+}
+
+// Segmentation of the chunk walks and the split of the SMs.
+//   G segments of L chunks per chain; fused: n_chain chain CTAs beside
+//   n_prep CTAs of two prep pipelines (one cooperative launch).
+struct TcPlan {
+    bool fused;
+    int G, L, n_chain, n_prep;
+    gdn::tc2::PrepOrder po;
+};
+
+// < 0: automatic; else the segments per chain (clamped to the chunk count)
+std::atomic<int> g_chain_segments{-1};
+
+// Fewest prep CTAs (two pipelines each) worth a fused launch: below this the
+// prep would lag the chains and two launches do better.
+constexpr int kMinFusedPrepCtas = 32;
+// Share of the SMs given to chain CTAs in a fused launch, in 1/16ths.
+constexpr int kChainShare16 = 6;
+// Fewest chunks per segment (a segment also walks back a few chunks first).
+constexpr int kMinSegChunks = 16;
+// Tail positions of every segment the prep produces first (the next
+// segment's walk back reads them before anything else).
+constexpr int kTailFirst = 12;
+
+TcPlan plan_tc(int chains, int nC, bool coop) {
+    const int sms = sm_count();
+    TcPlan p{};
+    p.fused = coop && chains + kMinFusedPrepCtas <= sms;
+    int G;
+    const int forced = g_chain_segments.load(std::memory_order_relaxed);
+    const int gmax = nC / kMinSegChunks > 1 ? nC / kMinSegChunks : 1;
+    if (forced > 0) {
+        G = forced;
+    } else if (p.fused) {
+        G = (sms * kChainShare16 / 16) / chains;
+        if (G > gmax) G = gmax;
+    } else {
+        G = sms / chains;
+        if (G > gmax) G = gmax;
+    }
+    if (G < 1) G = 1;
+    if (G > nC) G = nC;
+    p.L = (nC + G - 1) / G;
+    p.G = (nC + p.L - 1) / p.L;
+    p.n_chain = chains * p.G;
+    if (p.fused && p.n_chain + kMinFusedPrepCtas > sms) p.fused = false;
+    p.n_prep = p.fused ? sms - p.n_chain : 0;
+    p.po.G = p.G;
+    p.po.L = p.L;
+    p.po.tail = p.G > 1 ? (p.L < kTailFirst ? p.L : kTailFirst) : 0;
+    return p;
+}
+
 template <int DV>
 gdn_status launch_prep(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq, const CUtensorMap &mv,
-                       unsigned char *recs, int nC, int ndir, unsigned int *err) {
+                       unsigned char *recs, float *lb, int nC, int ndir, const gdn::tc2::PrepOrder &po,
+                       unsigned int *err) {
     using SM = gdn::tc2::PrepSmem<DV>;
     auto kern = gdn::tc2::prep_kernel<DV>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
@@ -295,21 +356,10 @@ gdn_status launch_prep(const Args &a, const CUtensorMap &mk, const CUtensorMap &
     const long long slots = (long long)sm_count() * gdn::tc2::kPrepCtasPerSm;
     const int grid = (int)(ntasks < slots ? ntasks : slots);
     gdn::LaunchScope ls("tc_prep", a.stream);
-    kern<<<grid, gdn::tc2::kPrepThreads, SM::kAlloc, a.stream>>>(mk, mq, mv, a.alpha, a.beta, recs, a.T,
-                                                                 a.H, nC, nbh, ndir, err);
+    kern<<<grid, gdn::tc2::kPrepThreads, SM::kAlloc, a.stream>>>(mk, mq, mv, a.alpha, a.beta, recs, lb, a.T, a.H, nC,
+                                                                 nbh, ndir, po, err);
     return launch_status();
 }
-
-// State columns per chain CTA: 32 while the grid still fits on the SMs (the
-// chain is then latency-bound and the narrower slice halves each step's
-// epilogues), else 64 (half the CTAs and half the record re-reads).
-int chain_slice_cols(int B, int H, int dv, int ndir) {
-    return (long long)B * H * ndir * (dv / 32) <= sm_count() ? 32 : 64;
-}
-
-// Fewest prep CTAs (two pipelines each) worth a fused launch: below this the
-// prep would lag the chains and two launches do better.
-constexpr int kMinFusedPrepCtas = 32;
 
 // o (bf16) <- sum (fp32), n a multiple of 4 elements.
 __global__ void cast_bf16_kernel(const float4 *__restrict__ sum, uint2 *__restrict__ o, size_t n4) {
@@ -322,61 +372,39 @@ __global__ void cast_bf16_kernel(const float4 *__restrict__ sum, uint2 *__restri
     }
 }
 
-// Output of a chain: target [B, T, H, DV] tensor of Tout (kOutStore) or fp32
-// (kOutPair, both directions adding up there).
-template <int DV, int NS, typename Tout>
-gdn_status launch_chain(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq,
-                        const unsigned char *recs, int nC, int ndir, const gdn::tc2::ChainStates &states,
-                        const gdn::tc2::ChainOut<Tout> &out, const void *target,
-                        unsigned int *err) {
-    using SM = gdn::tc2::ChainSmem<NS>;
-    const bool f32t = std::is_same<Tout, float>::value || out.mode == gdn::tc2::kOutPair;
-    CUtensorMap mo;
-    if (!encode_map(&mo, target, a.B, a.T, a.H, DV, f32t ? 32 : NS, (f32t || NS == 64) ? 128 : 64, f32t ? 4 : 2))
-        return GDN_ERR_CUDA;
-    auto kern = gdn::tc2::chain_kernel<DV, NS, Tout>;
+template <int DV, typename Tout>
+gdn_status launch_chain(const Args &a, const CUtensorMap &mo, const unsigned char *recs, int nC, int ndir,
+                        const gdn::tc2::ChainStates &states, const gdn::tc2::ChainOut<Tout> &out,
+                        const gdn::tc2::ChainSeg &seg, unsigned int *err) {
+    using SM = gdn::tc2::ChainSmem<DV>;
+    auto kern = gdn::tc2::chain_kernel<DV, Tout>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
         return GDN_ERR_CUDA;
     gdn::LaunchScope ls(ndir == 2 ? "tc_chain_bidir" : "tc_chain", a.stream);
-    kern<<<dim3(DV / NS, a.B * a.H, ndir), gdn::tc2::chain_threads<NS>(), SM::kAlloc, a.stream>>>(
-        mk, mq, mo, recs, states, out, a.T, a.H, nC, err);
+    kern<<<dim3(seg.G, a.B * a.H, ndir), gdn::tc2::kChainThreads, SM::kAlloc, a.stream>>>(mo, recs, states, out, seg,
+                                                                                          a.H, nC, err);
     return launch_status();
 }
 
-template <int DV, typename Tout>
-gdn_status launch_chain_ns(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq,
-                           const unsigned char *recs, int nC, int ndir, const gdn::tc2::ChainStates &states,
-                           const gdn::tc2::ChainOut<Tout> &out, const void *target,
-                           unsigned int *err) {
-    if (chain_slice_cols(a.B, a.H, DV, ndir) == 32)
-        return launch_chain<DV, 32, Tout>(a, mk, mq, recs, nC, ndir, states, out, target, err);
-    return launch_chain<DV, 64, Tout>(a, mk, mq, recs, nC, ndir, states, out, target, err);
-}
-
-// Prep and chain in one cooperative launch (tc_fused.cuh): n_chain chain CTAs
-// and n_prep CTAs of two prep pipelines each, all resident at once.  Returns
+// Prep and chain in one cooperative launch (tc_fused.cuh).  Returns
 // GDN_ERR_UNSUPPORTED (nothing launched) when the launch cannot be cooperative.
-template <int DV, int NS, typename Tout>
+template <int DV, typename Tout>
 gdn_status launch_fused(const Args &a, const CUtensorMap &mk, const CUtensorMap &mq, const CUtensorMap &mv,
-                        unsigned char *recs, unsigned int *ready, int nC, int ndir, int n_chain, int n_prep,
-                        const gdn::tc2::ChainStates &states, const gdn::tc2::ChainOut<Tout> &out,
-                        const void *target, unsigned int *err) {
-    const bool f32t = std::is_same<Tout, float>::value || out.mode == gdn::tc2::kOutPair;
-    CUtensorMap mo;
-    if (!encode_map(&mo, target, a.B, a.T, a.H, DV, f32t ? 32 : NS, (f32t || NS == 64) ? 128 : 64, f32t ? 4 : 2))
-        return GDN_ERR_CUDA;
-    auto kern = gdn::tc2::fused_kernel<DV, NS, Tout>;
-    constexpr int smem = gdn::tc2::fused_smem_alloc<DV, NS>();
-    constexpr int threads = gdn::tc2::chain_threads<NS>();
+                        const CUtensorMap &mo, unsigned char *recs, float *lb, unsigned int *ready, int nC, int ndir,
+                        const TcPlan &p, const gdn::tc2::ChainStates &states, const gdn::tc2::ChainOut<Tout> &out,
+                        const gdn::tc2::ChainSeg &seg, unsigned int *err) {
+    auto kern = gdn::tc2::fused_kernel<DV, Tout>;
+    constexpr int smem = gdn::tc2::fused_smem_alloc<DV>();
+    constexpr int threads = gdn::tc2::kChainThreads;
     static_assert(smem <= 227 * 1024, "fused launch shared memory");
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return GDN_ERR_CUDA;
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess ||
-        per_sm < 1 || n_chain + n_prep > per_sm * sm_count())
+        per_sm < 1 || p.n_chain + p.n_prep > per_sm * sm_count())
         return GDN_ERR_UNSUPPORTED;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(n_chain + n_prep);
+    cfg.gridDim = dim3(p.n_chain + p.n_prep);
     cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = a.stream;
@@ -386,8 +414,8 @@ gdn_status launch_fused(const Args &a, const CUtensorMap &mk, const CUtensorMap 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     gdn::LaunchScope ls("tc_fused", a.stream);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, mo, a.alpha, a.beta, recs, ready, states,
-                                             out, a.T, a.H, nC, a.B * a.H, ndir, n_chain, err);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, mo, a.alpha, a.beta, recs, lb, ready, states,
+                                             out, seg, p.po, a.T, a.H, nC, a.B * a.H, ndir, p.n_chain, err);
     if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorNotSupported) {
         (void)cudaGetLastError();
         return GDN_ERR_UNSUPPORTED;
@@ -412,10 +440,13 @@ gdn_status run_tc(const Args &a, int bidir) {
     if (!err) return GDN_ERR_CUDA;
     const int nC = (a.T + kChunk - 1) / kChunk;
     const int ndir = bidir ? 2 : 1;
+    const size_t nrec = (size_t)ndir * a.B * a.H * nC;
     unsigned char *recs = static_cast<unsigned char *>(a.ws);
-    unsigned char *p = recs + round_up((size_t)ndir * a.B * a.H * nC * tc_record_bytes(DV), 256);
+    unsigned char *p = recs + round_up(nrec * tc_record_bytes(DV), 256);
     unsigned int *ready = reinterpret_cast<unsigned int *>(p);
-    p += round_up((size_t)ndir * a.B * a.H * nC * sizeof(unsigned int), 256);
+    p += round_up(nrec * sizeof(unsigned int), 256);
+    float *lb = reinterpret_cast<float *>(p);
+    p += round_up(nrec * sizeof(float), 256);
     gdn::tc2::ChainOut<Tout> out{};
     constexpr bool f32_out = std::is_same<Tout, float>::value;
     void *target = a.o;
@@ -429,12 +460,14 @@ gdn_status run_tc(const Args &a, int bidir) {
         }
         out.mode = gdn::tc2::kOutPair;
         out.cnt = reinterpret_cast<unsigned int *>(p);
-        if (cudaMemsetAsync(out.cnt, 0, tc_pair_counters(a.B, a.T, a.H, DV) * sizeof(unsigned int), a.stream) !=
+        if (cudaMemsetAsync(out.cnt, 0, tc_pair_counters(a.B, a.T, a.H) * sizeof(unsigned int), a.stream) !=
             cudaSuccess)
             return GDN_ERR_CUDA;
     } else {
         out.mode = gdn::tc2::kOutStore;
     }
+    CUtensorMap mo;
+    if (!encode_out_map(&mo, target, a, DV, f32_out || bidir)) return GDN_ERR_CUDA;
     gdn::tc2::ChainStates states{};
     states.in[0] = a.state_in;
     states.out[0] = a.state_out;
@@ -443,25 +476,20 @@ gdn_status run_tc(const Args &a, int bidir) {
         states.out[1] = a.state_out_bwd;
     }
 
-    // One cooperative launch (prep on the SMs the chain leaves free) when the
-    // chain grid leaves room for it; else prep, then chain.
-    const int sms = sm_count();
-    const int ns = chain_slice_cols(a.B, a.H, DV, ndir);
-    const long long n_chain = (long long)(DV / ns) * a.B * a.H * ndir;
+    // One cooperative launch (prep on the SMs the chains leave free) when the
+    // chains leave room for it; else prep, then chain.
+    TcPlan plan = plan_tc(a.B * a.H * ndir, nC, cooperative_supported());
+    gdn::tc2::ChainSeg seg{plan.G, plan.L, lb};
     gdn_status s = GDN_ERR_UNSUPPORTED;
-    if (n_chain + kMinFusedPrepCtas <= sms && cooperative_supported()) {
-        if (cudaMemsetAsync(ready, 0, (size_t)ndir * a.B * a.H * nC * sizeof(unsigned int), a.stream) != cudaSuccess)
-            return GDN_ERR_CUDA;
-        const int n_prep = sms - (int)n_chain;
-        s = ns == 32 ? launch_fused<DV, 32, Tout>(a, mk, mq, mv, recs, ready, nC, ndir, (int)n_chain, n_prep, states,
-                                                  out, target, err)
-                     : launch_fused<DV, 64, Tout>(a, mk, mq, mv, recs, ready, nC, ndir, (int)n_chain, n_prep, states,
-                                                  out, target, err);
+    if (plan.fused) {
+        if (cudaMemsetAsync(ready, 0, nrec * sizeof(unsigned int), a.stream) != cudaSuccess) return GDN_ERR_CUDA;
+        s = launch_fused<DV, Tout>(a, mk, mq, mv, mo, recs, lb, ready, nC, ndir, plan, states, out, seg, err);
     }
     if (s == GDN_ERR_UNSUPPORTED) {
-        s = launch_prep<DV>(a, mk, mq, mv, recs, nC, ndir, err);
+        gdn::tc2::PrepOrder po{1, nC, 0};
+        s = launch_prep<DV>(a, mk, mq, mv, recs, lb, nC, ndir, po, err);
         if (s != GDN_OK) return s;
-        s = launch_chain_ns<DV, Tout>(a, mk, mq, recs, nC, ndir, states, out, target, err);
+        s = launch_chain<DV, Tout>(a, mo, recs, nC, ndir, states, out, seg, err);
     }
     if (s != GDN_OK || !bidir || f32_out) return s;
     gdn::LaunchScope ls("tc_bidir_cast", a.stream);
@@ -818,6 +846,10 @@ unsigned long long gdn_launch_count(void) {
 int gdn_set_short_call_tokens(int max_t) {
     const int v = max_t < 0 ? -1 : (max_t > gdn::tok::kMaxT ? gdn::tok::kMaxT : max_t);
     return g_short_call_tokens.exchange(v);
+}
+
+int gdn_set_chain_segments(int g) {
+    return g_chain_segments.exchange(g < 1 ? -1 : g);
 }
 
 void gdn_set_kernel_timing(int on) { gdn::LaunchStats::get().timing.store(on != 0); }

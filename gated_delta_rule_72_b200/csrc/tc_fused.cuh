@@ -1,16 +1,17 @@
 // tc_fused.cuh -- prep and chain in one cooperative launch.
 //
-// When the chain needs fewer CTAs than the GPU has SMs (few heads, long
-// sequences: the chain is latency-bound and most SMs would idle), one launch
-// runs both: CTAs [0, n_chain) are chain CTAs (one state slice each, as in
-// chain_kernel) and every other CTA runs two prep pipelines (each as in
-// prep_kernel, on half of the CTA's shared memory and TMEM).  The prep
-// pipelines walk the chunk tasks in the order the chains consume them and set
-// a ready flag per record once its stores have landed; a chain's loader waits
-// for the flag of each record before fetching it.  The launch is cooperative,
-// so every CTA is resident at once: the prep pipelines never wait on a chain,
-// and a chain only waits on prep pipelines that are running.  Every wait is
-// bounded (a flag wait gives up after kFlagWaitNs and flags an error).
+// When the chains need fewer CTAs than the GPU has SMs (few heads, long
+// sequences), one launch runs both: CTAs [0, n_chain) are chain CTAs (one
+// segment of one chain each, as in chain_kernel) and every other CTA runs two
+// prep pipelines (each as in prep_kernel, on half of the CTA's shared memory
+// and TMEM).  The prep pipelines walk the chunk tasks in the order the chains
+// consume them and set a ready flag per record once its stores have landed; a
+// chain waits for the flag of each record (and of each chunk bound it reads
+// while choosing its starting point) before using it.  The launch is
+// cooperative, so every CTA is resident at once: the prep pipelines never wait
+// on a chain, and a chain only waits on prep pipelines that are running.
+// Every wait is bounded (a flag wait gives up after kFlagWaitNs and flags an
+// error).
 #pragma once
 
 #include "tc_chain.cuh"
@@ -27,31 +28,30 @@ struct FusedPrepSmem {
     static constexpr int kBytes = kCtl + 16;
 };
 
-template <int DV, int NS>
+template <int DV>
 constexpr int fused_smem_alloc() {
-    return (ChainSmem<NS>::kAlloc > FusedPrepSmem<DV>::kBytes + 1024) ? ChainSmem<NS>::kAlloc
+    return (ChainSmem<DV>::kAlloc > FusedPrepSmem<DV>::kBytes + 1024) ? ChainSmem<DV>::kAlloc
                                                                        : FusedPrepSmem<DV>::kBytes + 1024;
 }
 
-// grid n_chain + n_prep CTAs (cooperative), block chain_threads<NS>().
-// Chain CTA i: slice i % (DV/NS), (b,h) (i / (DV/NS)) % nbh, direction i / (DV/NS * nbh).
-template <int DV, int NS, typename Tout>
-__global__ void __launch_bounds__(chain_threads<NS>(), 1)
+// grid n_chain + n_prep CTAs (cooperative), block kChainThreads.
+// Chain CTA i: segment i % G, (b,h) (i / G) % nbh, direction i / (G * nbh).
+template <int DV, typename Tout>
+__global__ void __launch_bounds__(kChainThreads, 1)
 fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
              const float *__restrict__ alpha, const float *__restrict__ beta, unsigned char *__restrict__ recs,
-             unsigned int *__restrict__ ready, const ChainStates states,
-             const ChainOut<Tout> out, int T, int H, int nC, int nbh, int ndir, int n_chain,
-             unsigned int *__restrict__ err)
+             float *__restrict__ lb, unsigned int *__restrict__ ready, const ChainStates states,
+             const ChainOut<Tout> out, const ChainSeg seg, PrepOrder po, int T, int H, int nC, int nbh, int ndir,
+             int n_chain, unsigned int *__restrict__ err)
 {
-    static_assert(chain_threads<NS>() >= 2 * kPrepThreads, "two prep pipelines per CTA");
+    static_assert(kChainThreads >= 2 * kPrepThreads, "two prep pipelines per CTA");
     extern __shared__ __align__(16) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const int nsl = DV / NS;
     if ((int)blockIdx.x < n_chain) {
         const int i = blockIdx.x;
-        chain_body<DV, NS, Tout>(&tm_k, &tm_q, &tm_o, recs, states, out, ready, T, H, nC, i % nsl,
-                                 (i / nsl) % nbh, i / (nsl * nbh), nsl, nbh, smem, err);
+        chain_body<DV, Tout>(&tm_o, recs, states, out, seg, ready, H, nC, i % seg.G, (i / seg.G) % nbh,
+                             i / (seg.G * nbh), nbh, smem, err);
         return;
     }
     // ---- two prep pipelines: warps 0-7 and 8-15 (the rest of the block idles)
@@ -69,7 +69,7 @@ fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     if (warp < 16) {
         const int pipe = warp >> 3;
         const int npipes = 2 * ((int)gridDim.x - n_chain);
-        prep_pipeline<DV>(&tm_k, &tm_q, &tm_v, alpha, beta, recs, ready, T, H, nC, nbh, ndir,
+        prep_pipeline<DV>(&tm_k, &tm_q, &tm_v, alpha, beta, recs, lb, ready, T, H, nC, nbh, ndir, po,
                           2 * ((int)blockIdx.x - n_chain) + pipe, npipes, smem + pipe * FS::kArea,
                           tmem + pipe * kPrepTmemCols, threadIdx.x & (kPrepThreads - 1), 1 + pipe, err);
     }

@@ -1,38 +1,31 @@
 // tc_prep.cuh -- chunk preparation on the tensor cores (tcgen05 + TMA).
 //
 // For every chunk of 64 tokens of every (b, h) and direction (fully
-// parallel; a persistent grid of two CTAs per SM walks the tasks and fetches
-// the next task's tiles with TMA while it finishes the current one) this kernel
-// computes, in the chunk's processing order r = 0..63 (the reverse direction
-// walks a chunk back to front):
+// parallel; a persistent grid of two pipelines per SM walks the tasks and
+// fetches the next task's tiles with TMA while it finishes the current one)
+// this kernel computes, in the chunk's processing order r = 0..63 (the
+// reverse direction walks a chunk back to front):
 //   g_r = sum_{m<=r} log alpha_m                          (prefix sum, fp32)
-//   [K; Q] K^T                                            (kind::f16, M=128, exact)
+//   [K; Q] K^T                                            (kind::f16 bf16, M=128, exact)
 //   L_rs = beta_r e^{g_r-g_s} (KK^T)_rs, s < r             (fp32)
 //   P_rs = e^{g_r-g_s} (QK^T)_rs, s <= r   (forward)     | readout mask
 //        = e^{g_{r-1}-g_s} (QK^T)_rs, s < r (reverse)    |
 //   T = (I + L)^{-1}                                      (blocked 16x16, CUDA cores)
-//   W = T diag(beta e^g) K,  U = T diag(beta) V           (kind::f16; the T of U as a
-//                                                          hi/lo pair, W rounds to bf16 anyway)
-//   dq_r = e^{g_r} (reverse: e^{g_{r-1}}),  dkk_r = e^{g_63 - g_r},  ds = e^{g_63}
-// and writes them as one record (tc_common.cuh) with rows in forward token
-// order: for the reverse direction every row and column index is mirrored
-// (r -> 63 - r), so that the chain kernel never needs to know the direction.
+//   W = T diag(beta e^g) K,  U = T diag(beta) V           (kind::f16 fp16, single-rounded T)
+//   Q~_r = dq_r q_r, dq_r = e^{g_r} (reverse: e^{g_{r-1}});  K~_r = e^{g_63 - g_r} k_r
+//   ds = e^{g_63}
+// and writes them as one fp16 record (tc_common.cuh) with rows in forward
+// token order: for the reverse direction every row and column index is
+// mirrored (r -> 63 - r), so that the chain kernel never needs to know the
+// direction.  Beside the record it writes the log of a bound on the 2-norm of
+// the chunk's state map, g_63 + sum_r ln max(1, |1 - beta_r |k_r|^2|), which
+// the chain uses to decide where a segment may start from a zero state.
 #pragma once
 
 #include "tc_common.cuh"
 
 namespace gdn {
 namespace tc2 {
-
-#ifdef GDN_PREP_TIMING
-// Development aid (not built into the library): cycle stamps of CTA 0's
-// tasks 2..11, thread 0.
-__device__ long long g_prep_ts[10][12];
-#define PREP_TS(slot) do { if (first_task == 0 && tid == 0 && (t / task_stride) >= 2 && (t / task_stride) < 12) \
-    g_prep_ts[t / task_stride - 2][slot] = clock64(); } while (0)
-#else
-#define PREP_TS(slot) do { } while (0)
-#endif
 
 template <int DV>
 struct PrepSmem {
@@ -42,18 +35,18 @@ struct PrepSmem {
     static constexpr int kL = kStage;                 // [64][65] fp32
     static constexpr int kT = kL + 64 * 65 * 4;       // [64][65] fp32
     static constexpr int kX = kT + 64 * 65 * 4;       // 3 x [16][16] fp32
-    static constexpr int kT1 = (kX + 3 * 256 * 4 + 1023) / 1024 * 1024;   // bf16 K-major 64 x 64
-    static constexpr int kT2h = kT1 + 8192;
-    static constexpr int kT2l = kT2h + 8192;
-    static constexpr int kGate = kT2l + 8192;         // g, beta, dq, dkk, beta e^g
-    static constexpr int kBar = kGate + 5 * 256;      // tma, mma, gram
+    static constexpr int kT1 = (kX + 3 * 256 * 4 + 1023) / 1024 * 1024;   // fp16 K-major 64 x 64
+    static constexpr int kT2 = kT1 + 8192;
+    static constexpr int kGate = kT2 + 8192;          // g, beta, dq, dkk, beta e^g
+    static constexpr int kMisc = kGate + 5 * 256;     // key-norm partials [2], record gate [4]
+    static constexpr int kBar = kMisc + 32;           // tma, mma, gram
     static constexpr int kCtl = kBar + 32;            // tmem base, abort, ds
     static constexpr int kBytes = kCtl + 16;
     static constexpr int kAlloc = kBytes + 1024;
     static_assert(kStage % 1024 == 0 && kT1 % 1024 == 0, "swizzled areas stay 1024-aligned");
-    // record staging: P and W images over T1 | T2h, U over L | T, gates over T2l
-    static_assert(kT2h == kT1 + 8192 && 64 * DV * 4 <= 2 * 64 * 65 * 4, "record staging areas");
-    static_assert(kAlloc <= 232448 / 2 - 1024, "two CTAs per SM");
+    // record staging: P and W images over T1 | T2, U over L | T
+    static_assert(64 * DV * 2 <= 2 * 64 * 65 * 4, "record staging areas");
+    static_assert(kAlloc <= 232448 / 2 - 1024, "two pipelines per SM");
 };
 
 constexpr int kPrepThreads = 256;
@@ -64,19 +57,40 @@ constexpr uint32_t kPrepColW = 0;      // M=64 x 128
 constexpr uint32_t kPrepColU = 128;    // M=64 x DV
 constexpr uint32_t kPrepTmemCols = 256;
 
+// Order of the prep tasks.  The chains of a launch are cut into G segments
+// of L chunks (walk order); a segment first walks back into the tail of the
+// segment before it.  So the tasks come position by position within the
+// segments, the last `tail` positions first (from the end backwards), then
+// the rest from the front; within a position: segment, direction, (b, h).
+struct PrepOrder {
+    int G, L, tail;
+};
+
+__device__ __forceinline__ bool prep_task(const PrepOrder &po, int t, int nbh, int ndir, int nC, int &dir,
+                                          int &c, int &bh) {
+    const int per = nbh * ndir * po.G;
+    const int j = t / per, rem = t - j * per;
+    bh = rem % nbh;
+    dir = (rem / nbh) % ndir;
+    const int g = rem / (nbh * ndir);
+    const int p = j < po.tail ? po.L - 1 - j : j - po.tail;
+    const int w = g * po.L + p;
+    c = dir == 0 ? w : nC - 1 - w;
+    return w < nC;
+}
+
 // One prep pipeline: 256 threads (ptid 0..255) with their own 1024-aligned
 // shared-memory area `smem` (PrepSmem<DV>), 256 TMEM columns from `tmem` and
 // named barrier `bar_id`; it walks tasks first_task, first_task + stride, ...
-// Tasks are ordered the way the chain consumes them: step k holds chunk k of
-// the causal direction and chunk nC-1-k of the reverse one, then (b, h).
-// With `ready` non-null, each record's flag is set (release) once its bulk
-// stores have landed, for a chain kernel that runs alongside.
+// (po order).  With `ready` non-null, each record's flag is set (release) once
+// its stores have landed, for a chain kernel that runs alongside.
 template <int DV>
 __device__ __forceinline__ void prep_pipeline(
     const CUtensorMap *tm_k, const CUtensorMap *tm_q, const CUtensorMap *tm_v,
     const float *__restrict__ alpha, const float *__restrict__ beta, unsigned char *__restrict__ recs,
-    unsigned int *__restrict__ ready, int T, int H, int nC, int nbh, int ndir, int first_task,
-    int task_stride, unsigned char *smem, uint32_t tmem, int ptid, int bar_id, unsigned int *__restrict__ err)
+    float *__restrict__ lb, unsigned int *__restrict__ ready, int T, int H, int nC, int nbh, int ndir,
+    PrepOrder po, int first_task, int task_stride, unsigned char *smem, uint32_t tmem, int ptid, int bar_id,
+    unsigned int *__restrict__ err)
 {
     using SM = PrepSmem<DV>;
     using RC = Rec<DV>;
@@ -88,6 +102,8 @@ __device__ __forceinline__ void prep_pipeline(
     float *dq_s = g_s + 128;
     float *dkk_s = g_s + 192;
     float *bg_s = g_s + 256;
+    float *kf_s = reinterpret_cast<float *>(smem + SM::kMisc);        // [2] key-norm terms
+    float *rgate_s = reinterpret_cast<float *>(smem + SM::kMisc + 16); // [4] record gate (ds)
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + SM::kBar);
     uint64_t *mma_bar = tma_bar + 1;
     uint64_t *g_bar = tma_bar + 2;     // the two K halves of the Gram product
@@ -99,7 +115,7 @@ __device__ __forceinline__ void prep_pipeline(
     const int half = warp >> 2;                    // column half handled by this warp
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t sbase = smem_u32(smem);
-    const int ntasks = ndir * nC * nbh;
+    const int ntasks = po.L * po.G * ndir * nbh;
     auto psync = [&]() { asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory"); };
 
     if (tid == 0) {
@@ -114,15 +130,15 @@ __device__ __forceinline__ void prep_pipeline(
     }
     psync();
 
-    auto task_of = [&](int t, int &dir, int &c, int &bh) {
-        bh = t % nbh;
-        const int k = t / (nbh * ndir);
-        dir = (t / nbh) % ndir;
-        c = dir == 0 ? k : nC - 1 - k;
+    // the next task of this pipeline with a chunk to prepare (ntasks if none)
+    auto next_valid = [&](int t) {
+        int dir, c, bh;
+        while (t < ntasks && !prep_task(po, t, nbh, ndir, nC, dir, c, bh)) t += task_stride;
+        return t;
     };
     auto issue_tma = [&](int t) {
         int dir, c, bh;
-        task_of(t, dir, c, bh);
+        prep_task(po, t, nbh, ndir, nC, dir, c, bh);
         const int b = bh / H, h = bh % H, t0 = c * 64;
         unsigned char *st = smem;
         mbar_arrive_expect_tx(tma_bar, SM::kStage);
@@ -140,39 +156,40 @@ __device__ __forceinline__ void prep_pipeline(
             if (err) atomicAdd(err, 1u);
         }
     };
-    // gates of a task, processing order: thread r < 64 loads row r
-    auto load_gates = [&](int t, float &la, float &bt) {
+    // gates of a task, processing order: thread r < 64 loads row r (raw alpha:
+    // the logarithm is taken when the value is used, so the load's latency is
+    // not waited for here)
+    auto load_gates = [&](int t, float &al, float &bt) {
         int dir, c, bh;
-        task_of(t, dir, c, bh);
+        prep_task(po, t, nbh, ndir, nC, dir, c, bh);
         const int b = bh / H, h = bh % H;
         const int tok = token_of_row(c, tid, dir);
         const size_t off = ((size_t)b * T + tok) * H + h;
-        la = tok < T ? __logf(alpha[off]) : 0.f;
+        al = tok < T ? alpha[off] : 1.f;
         bt = tok < T ? beta[off] : 0.f;
     };
 
-    int t = first_task;
+    int t = next_valid(first_task);
     if (t < ntasks && tid == 0) issue_tma(t);
-    float la_n = 0.f, bt_n = 0.f;
-    if (t < ntasks && tid < 64) load_gates(t, la_n, bt_n);
+    float al_n = 1.f, bt_n = 0.f;
+    if (t < ntasks && tid < 64) load_gates(t, al_n, bt_n);
     uint32_t tma_phase = 0, mma_phase = 0, g_phase = 0;
     unsigned int *pending_flag = nullptr;   // thread 0: ready flag of the last record stored
     const uint32_t st_addr = sbase;
 
-    for (; t < ntasks; t += task_stride) {
+    while (t < ntasks) {
         int dir, c, bh;
-        task_of(t, dir, c, bh);
+        prep_task(po, t, nbh, ndir, nC, dir, c, bh);
         const bool rev = dir != 0;
-        unsigned char *rec = recs + ((size_t)(dir * nbh + bh) * nC + c) * RC::kBytes;
-        const int tn = t + task_stride;
+        unsigned char *rec = recs + ((size_t)(dir * nbh + bh) * nC + c) * RC::kStride;
+        const int tn = next_valid(t + task_stride);
 
-        if (tid < 64) { g_s[tid] = la_n; beta_s[tid] = bt_n; }
+        if (tid < 64) { g_s[tid] = __logf(al_n); beta_s[tid] = bt_n; }
         wait_all(tma_bar, tma_phase);
         tma_phase ^= 1;
         psync();
-        PREP_TS(0);
         if (*abort_s) break;
-        if (tn < ntasks && tid < 64) load_gates(tn, la_n, bt_n);   // next task's gates travel meanwhile
+        if (tn < ntasks && tid < 64) load_gates(tn, al_n, bt_n);   // next task's gates travel meanwhile
         if (warp == 0) {  // inclusive prefix sum of log alpha, 2 rows per lane
             const float a0 = g_s[2 * lane], a1 = g_s[2 * lane + 1];
             float s = a0 + a1;
@@ -239,11 +256,10 @@ __device__ __forceinline__ void prep_pipeline(
         }
         wait_all(g_bar, g_phase);
         g_phase ^= 1;
-        PREP_TS(2);
         tc_fence_after();
         psync();  // gate vectors ready
-        PREP_TS(1);
-        // ---- L (fp32, to shared) and P (hi/lo images, staged for a bulk store) -------
+        // ---- L (fp32, to shared), P (fp16 image, staged for a bulk store) and the
+        //      key-norm term of the state map's bound --------------------------------
         {
             float G[32];
             {
@@ -256,7 +272,6 @@ __device__ __forceinline__ void prep_pipeline(
 #pragma unroll
                 for (int e = 0; e < 32; ++e) G[e] += G2[e];
             }
-            PREP_TS(9);
             const int ln = quarter * 32 + lane;          // TMEM lane = Gram row
             const int fl = ln & 63;                      // forward row within the chunk
             const int r = rev ? 63 - fl : fl;            // processing row
@@ -268,11 +283,19 @@ __device__ __forceinline__ void prep_pipeline(
             if (ln < 64) {
                 const float br = beta_s[r], gr = g_s[r];
                 const float eA = br * Xsm[64 + r * 4 + kA], eB = br * Xsm[64 + r * 4 + kB];
+                float kk = 0.f;                          // |k_r|^2 (diagonal of the Gram)
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int s = rev ? 63 - (f0 + e) : f0 + e;
                     const float w = fast ? (e < 16 ? eA : eB) * facs[s] : br * __expf(gr - g_s[s]);
                     Lsm[r * 65 + s] = s < r ? w * G[e] : 0.f;
+                    if (f0 + e == fl) kk = G[e];
+                }
+                if (half == (fl >> 5)) {   // warps 0 and 5 hold the diagonal of rows 0-31 / 32-63
+                    float term = __logf(fmaxf(1.f, fabsf(1.f - br * kk)));
+#pragma unroll
+                    for (int d = 16; d > 0; d >>= 1) term += __shfl_xor_sync(0xffffffffu, term, d);
+                    if (lane == 0) kf_s[half] = term;
                 }
             } else {
                 const float gq = rev ? (r > 0 ? g_s[r - 1] : 0.f) : g_s[r];
@@ -288,27 +311,26 @@ __device__ __forceinline__ void prep_pipeline(
                         const float w = fast ? (cc < 2 ? eA : eB) * facs[s] : __expf(gq - g_s[s]);
                         v[e] = keep ? w * G[cc * 8 + e] : 0.f;
                     }
-                    uint4 hi, lo;
-                    split2(v[0], v[1], hi.x, lo.x);
-                    split2(v[2], v[3], hi.y, lo.y);
-                    split2(v[4], v[5], hi.z, lo.z);
-                    split2(v[6], v[7], hi.w, lo.w);
-                    const int off = sw128(fl, f0 + cc * 8, 0);
-                    *reinterpret_cast<uint4 *>(smem + SM::kT1 + off) = hi;          // the record's
-                    *reinterpret_cast<uint4 *>(smem + SM::kT1 + 8192 + off) = lo;   // P_hi | P_lo
+                    uint4 p;
+                    p.x = pack_f16(v[0], v[1]); p.y = pack_f16(v[2], v[3]);
+                    p.z = pack_f16(v[4], v[5]); p.w = pack_f16(v[6], v[7]);
+                    *reinterpret_cast<uint4 *>(smem + SM::kT1 + sw128(fl, f0 + cc * 8, 0)) = p;
                 }
                 fence_async_shared();
             }
         }
-        PREP_TS(10);
         tc_fence_before();
         psync();
         if (tid == 0) {
-            bulk_store(rec + RC::kPh, smem + SM::kT1, 16384);
+            bulk_store(rec + RC::kP, smem + SM::kT1, 8192);
             bulk_commit_group();
+            lb[(size_t)(dir * nbh + bh) * nC + c] = g_s[63] + kf_s[0] + kf_s[1];
+            rgate_s[0] = *ds_s;
+            rgate_s[1] = rgate_s[2] = rgate_s[3] = 0.f;
         }
-        PREP_TS(3);
-        // ---- T = (I + L)^{-1}, blocked 16 x 16 (processing order) ------------------
+        // ---- T = (I + L)^{-1}, blocked 16 x 16 (processing order); meanwhile the
+        //      other threads turn the tiles into fp16: K and V in place (operands of
+        //      W and U), Q~ and K~ straight into the record -----------------------
         if (tid < 64) {
             const int blk = tid >> 4, j = tid & 15, o0 = blk * 16;
             float x[16];
@@ -326,9 +348,39 @@ __device__ __forceinline__ void prep_pipeline(
                 const int i = e >> 6, jj = e & 63;
                 if ((jj >> 4) > (i >> 4)) Tsm[i * 65 + jj] = 0.f;
             }
+            // 16-byte chunks: K blocks (2 x 512), Q blocks (2 x 512), V blocks (DV/64 x 512)
+            constexpr int kChunks = 2048 + (DV / 64) * 512;
+            for (int i = tid - 64; i < kChunks; i += kPrepThreads - 64) {
+                const int blk = i >> 9, within = (i & 511) * 16, f = (i & 511) >> 3;
+                const int rr = rev ? 63 - f : f;
+                unsigned char *src;
+                if (blk < 2) src = smem + blk * 16384 + within;                    // K
+                else if (blk < 4) src = smem + (blk - 2) * 16384 + 8192 + within;  // Q
+                else src = smem + SM::kKQ + (blk - 4) * 8192 + within;            // V
+                const uint4 raw = *reinterpret_cast<const uint4 *>(src);
+                const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
+                uint32_t o16[4], sc16[4];
+                const float scale = blk < 2 ? dkk_s[rr] : dq_s[rr];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x2 = unpack_bf16(in[e]);
+                    o16[e] = pack_f16(x2.x, x2.y);
+                    sc16[e] = pack_f16(scale * x2.x, scale * x2.y);
+                }
+                if (blk < 2) {
+                    *reinterpret_cast<uint4 *>(src) = make_uint4(o16[0], o16[1], o16[2], o16[3]);
+                    *reinterpret_cast<uint4 *>(rec + RC::kK + blk * 8192 + within) =
+                        make_uint4(sc16[0], sc16[1], sc16[2], sc16[3]);
+                } else if (blk < 4) {
+                    *reinterpret_cast<uint4 *>(rec + RC::kQW + (blk - 2) * 16384 + within) =
+                        make_uint4(sc16[0], sc16[1], sc16[2], sc16[3]);
+                } else {
+                    *reinterpret_cast<uint4 *>(src) = make_uint4(o16[0], o16[1], o16[2], o16[3]);
+                }
+            }
+            __threadfence();   // the record's Q~ and K~ are published with its flag
         }
         psync();
-        PREP_TS(4);
         // off-diagonal blocks by bands: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj, i = j + band,
         // each thread a 2 x 2 tile (independent accumulators, conflict-free loads)
         for (int band = 1; band < 4; ++band) {
@@ -369,9 +421,8 @@ __device__ __forceinline__ void prep_pipeline(
         // the P store has read its staging area (the T images go there next)
         if (tid == 0) bulk_wait_read_all();
         psync();
-        PREP_TS(5);
-        // ---- A operands T diag(beta e^g) (bf16) and T diag(beta) (hi/lo pair), in
-        //      forward row/column order (mirrored for the reverse direction) --------
+        // ---- A operands T diag(beta e^g) and T diag(beta) (fp16), in forward
+        //      row/column order (mirrored for the reverse direction) ------------------
         for (int cell = tid; cell < 64 * 8; cell += kPrepThreads) {
             const int fr = cell & 63, fc0 = (cell >> 6) * 8;
             const int r = rev ? 63 - fr : fr;
@@ -383,44 +434,38 @@ __device__ __forceinline__ void prep_pipeline(
                 a[e] = tv * bg_s[s];
                 bvals[e] = tv * beta_s[s];
             }
-            uint4 h1, h2, l2;
-            h1.x = pack_bf16(a[0], a[1]); h1.y = pack_bf16(a[2], a[3]);
-            h1.z = pack_bf16(a[4], a[5]); h1.w = pack_bf16(a[6], a[7]);
-            split2(bvals[0], bvals[1], h2.x, l2.x); split2(bvals[2], bvals[3], h2.y, l2.y);
-            split2(bvals[4], bvals[5], h2.z, l2.z); split2(bvals[6], bvals[7], h2.w, l2.w);
+            uint4 h1, h2;
+            h1.x = pack_f16(a[0], a[1]); h1.y = pack_f16(a[2], a[3]);
+            h1.z = pack_f16(a[4], a[5]); h1.w = pack_f16(a[6], a[7]);
+            h2.x = pack_f16(bvals[0], bvals[1]); h2.y = pack_f16(bvals[2], bvals[3]);
+            h2.z = pack_f16(bvals[4], bvals[5]); h2.w = pack_f16(bvals[6], bvals[7]);
             const int off = kmaj64(fr, fc0);
             *reinterpret_cast<uint4 *>(smem + SM::kT1 + off) = h1;
-            *reinterpret_cast<uint4 *>(smem + SM::kT2h + off) = h2;
-            *reinterpret_cast<uint4 *>(smem + SM::kT2l + off) = l2;
+            *reinterpret_cast<uint4 *>(smem + SM::kT2 + off) = h2;
         }
         fence_async_shared();
         psync();
-        PREP_TS(6);
-        // ---- W = T1 K and U = T2 V on the tensor cores (K and V straight from the tiles)
+        // ---- W = T1 K and U = T2 V on the tensor cores (fp16 K and V in the tiles)
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t idw = idesc(64, 128, 1, 0, 1);
-            constexpr uint32_t idu = idesc(64, DV, 1, 0, 1);
+            constexpr uint32_t idw = idesc(64, 128, 0, 0, 1);
+            constexpr uint32_t idu = idesc(64, DV, 0, 0, 1);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
                 mma_bf16(tmem + kPrepColW, sdesc_noswz(sbase + SM::kT1 + 2 * s * 1024, 1024, 128),
                          sdesc_sw128_mn(st_addr + s * 2048, 16384), idw, s > 0);
-                const uint64_t bv = sdesc_sw128_mn(st_addr + SM::kKQ + s * 2048, 8192);
-                mma_bf16(tmem + kPrepColU, sdesc_noswz(sbase + SM::kT2h + 2 * s * 1024, 1024, 128),
-                         bv, idu, s > 0);
-                mma_bf16(tmem + kPrepColU, sdesc_noswz(sbase + SM::kT2l + 2 * s * 1024, 1024, 128),
-                         bv, idu, 1);
+                mma_bf16(tmem + kPrepColU, sdesc_noswz(sbase + SM::kT2 + 2 * s * 1024, 1024, 128),
+                         sdesc_sw128_mn(st_addr + SM::kKQ + s * 2048, 8192), idu, s > 0);
             }
             mma_commit(mma_bar);
         }
         wait_all(mma_bar, mma_phase);
-        PREP_TS(7);
         mma_phase ^= 1;
         tc_fence_after();
         // the tiles are consumed: fetch the next task's while this one is written out
         if (tn < ntasks && tid == 0) issue_tma(tn);
-        // ---- record: W image, U granules and gate vectors, staged in the areas the
-        //      products are done with (T images, L/T) and written by bulk stores -------
+        // ---- record: W image and U rows (fp16), staged in the areas the products
+        //      are done with (T images, L/T) and written by bulk stores ---------------
         {
             const bool row_lane = lane < 16;
             const int f = quarter * 16 + lane;       // forward row (M=64 accumulator layout)
@@ -433,8 +478,8 @@ __device__ __forceinline__ void prep_pipeline(
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         uint4 p;
-                        p.x = pack_bf16(w[8 * q], w[8 * q + 1]); p.y = pack_bf16(w[8 * q + 2], w[8 * q + 3]);
-                        p.z = pack_bf16(w[8 * q + 4], w[8 * q + 5]); p.w = pack_bf16(w[8 * q + 6], w[8 * q + 7]);
+                        p.x = pack_f16(w[8 * q], w[8 * q + 1]); p.y = pack_f16(w[8 * q + 2], w[8 * q + 3]);
+                        p.z = pack_f16(w[8 * q + 4], w[8 * q + 5]); p.w = pack_f16(w[8 * q + 6], w[8 * q + 7]);
                         *reinterpret_cast<uint4 *>(smem + SM::kT1 + sw128(f, half * 64 + 8 * q, 8192)) = p;
                     }
                 }
@@ -446,22 +491,14 @@ __device__ __forceinline__ void prep_pipeline(
                 tmem_ld16(tmem + lane_base + kPrepColU + col, u);
                 tmem_ld16(tmem + lane_base + kPrepColU + col + 16, u + 16);
                 tmem_wait_ld();
-                if (row_lane) {   // granule col/32, row f
-                    unsigned char *sl = smem + SM::kL + (col / kSliceCols) * RC::kUSlice;
+                if (row_lane) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        *reinterpret_cast<float4 *>(sl + u_off(f, 4 * i)) =
-                            make_float4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
-                }
-            }
-            if (tid < 64) {
-                const int r = rev ? 63 - tid : tid;   // record row tid <- processing row r
-                float *gate = reinterpret_cast<float *>(smem + SM::kT2l);
-                gate[tid] = dq_s[r];
-                gate[64 + tid] = dkk_s[r];
-                if (tid == 0) {
-                    gate[128] = *ds_s;
-                    gate[129] = gate[130] = gate[131] = 0.f;
+                    for (int i = 0; i < 4; ++i) {
+                        uint4 p;
+                        p.x = pack_f16(u[8 * i], u[8 * i + 1]); p.y = pack_f16(u[8 * i + 2], u[8 * i + 3]);
+                        p.z = pack_f16(u[8 * i + 4], u[8 * i + 5]); p.w = pack_f16(u[8 * i + 6], u[8 * i + 7]);
+                        *reinterpret_cast<uint4 *>(smem + SM::kL + u16_off<DV>(f, col + 8 * i)) = p;
+                    }
                 }
             }
             fence_async_shared();
@@ -469,12 +506,13 @@ __device__ __forceinline__ void prep_pipeline(
         tc_fence_before();
         psync();
         if (tid == 0) {
-            bulk_store(rec + RC::kW, smem + SM::kT1, 16384);
-            bulk_store(rec + RC::kU, smem + SM::kL, 64 * DV * 4);
-            bulk_store(rec + RC::kGate, smem + SM::kT2l, RC::kGateCopy);
+            bulk_store(rec + RC::kQW + 8192, smem + SM::kT1, 8192);              // W, d_k 0-63
+            bulk_store(rec + RC::kQW + 16384 + 8192, smem + SM::kT1 + 8192, 8192);   // W, d_k 64-127
+            bulk_store(rec + RC::kU, smem + SM::kL, 64 * DV * 2);
+            bulk_store(rec + RC::kGate, rgate_s, 16);
             bulk_commit_group();
         }
-        PREP_TS(8);
+        t = tn;
     }
 
     if (tid == 0) {
@@ -499,8 +537,8 @@ template <int DV>
 __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
 prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
             const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ alpha,
-            const float *__restrict__ beta, unsigned char *__restrict__ recs, int T, int H,
-            int nC, int nbh, int ndir, unsigned int *__restrict__ err)
+            const float *__restrict__ beta, unsigned char *__restrict__ recs, float *__restrict__ lb, int T, int H,
+            int nC, int nbh, int ndir, PrepOrder po, unsigned int *__restrict__ err)
 {
     using SM = PrepSmem<DV>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -514,7 +552,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_s;
-    prep_pipeline<DV>(&tm_k, &tm_q, &tm_v, alpha, beta, recs, nullptr, T, H, nC, nbh, ndir, blockIdx.x,
+    prep_pipeline<DV>(&tm_k, &tm_q, &tm_v, alpha, beta, recs, lb, nullptr, T, H, nC, nbh, ndir, po, blockIdx.x,
                       gridDim.x, smem, tmem, threadIdx.x, 0, err);
     __syncthreads();
     if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, kPrepTmemCols);

@@ -198,6 +198,23 @@ GDN_API size_t gdn_workspace_size(int B, int T, int H, int dk, int dv, gdn_dtype
 GDN_API int gdn_set_short_call_tokens(int max_t);
 
 /*
+ * gdn_set_chain_segments -- how many segments the tensor-core path cuts each
+ * (b, h, direction) chunk walk into (sequence parallelism; bf16 inputs with
+ * d_k = 128).  g < 1: automatic (the default): enough segments to occupy the
+ * SMs, at least 16 chunks each; g >= 1: g segments (at most one per chunk).
+ * A segment other than the first starts from a zero state some chunks before
+ * its first output, at the first chunk boundary where the 2-norm bound of the
+ * skipped state maps, the product over the skipped tokens of
+ * alpha_t max(1, |1 - beta_t |k_t|^2|), falls to 2^-30 (or from the true
+ * initial state if the walk back reaches the start).  The state dropped there
+ * reaches the segment's first output scaled by at most 2^-30, so results
+ * agree with one segment up to rounding; only the speed depends on how fast
+ * the gates forget.  Returns the previous setting (-1 for automatic).
+ * Process-wide, read at each call; the workspace does not depend on it.
+ */
+GDN_API int gdn_set_chain_segments(int g);
+
+/*
  * gdn_vda_scan -- the frame-wise delta operator: the sequence is F frames of
  * U consecutive tokens (T = F * U) and the state is written once per frame,
  * by all of the frame's tokens at once:

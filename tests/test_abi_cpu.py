@@ -156,6 +156,19 @@ def test_short_call_threshold_is_clamped(lib):
         lib.gdn_set_short_call_tokens(prev)
 
 
+def test_chain_segment_setting_round_trips(lib):
+    """gdn_set_chain_segments: values below 1 mean automatic (-1, the
+    default); returns the previous setting (host-side only)."""
+    prev = lib.gdn_set_chain_segments(4)
+    try:
+        assert lib.gdn_set_chain_segments(0) == 4
+        assert lib.gdn_set_chain_segments(-3) == -1
+        assert lib.gdn_set_chain_segments(7) == -1
+        assert lib.gdn_set_chain_segments(7) == 7
+    finally:
+        lib.gdn_set_chain_segments(prev)
+
+
 def _bidir_states(**kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, alpha=FAKE, beta=FAKE, state_in=None, state_in_bwd=None,
              state_out=None, state_out_bwd=None, o=FAKE, B=1, T=64, H=2, dk=64, dv=64, dt=0, o_dt=0,

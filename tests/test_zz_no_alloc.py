@@ -6,12 +6,13 @@ inside libgdn.so instead of a caller workspace.
 
 Called through the C-ABI, two calls in a row must match the ordinary
 gdn_step on the same inputs, within the bf16-input tolerance the other
-parity tests use.  This file is collected last on purpose."""
+parity tests use, and on a sampled head the FP64 oracle run over both
+calls' tokens.  This file is collected last on purpose."""
 import pytest
 import torch
 
 from gated_delta_rule_72_b200 import _lib, inputs
-from tests.gpu_util import TOL, rel_err
+from tests.gpu_util import TOL, oracle_heads, rel_err
 
 
 @pytest.mark.gpu
@@ -26,6 +27,7 @@ def test_noalloc_step_matches_step_on_two_calls():
     st_ref = torch.zeros(B, H, dk, dv, device="cuda")
     st_new = torch.zeros(B, H, dk, dv, device="cuda")
     stream = torch.cuda.current_stream().cuda_stream
+    outs = []
     for call in range(2):
         sl = slice(call * T, (call + 1) * T)
         x = {n: t[:, sl].contiguous() for n, t in d.items()}
@@ -43,3 +45,9 @@ def test_noalloc_step_matches_step_on_two_calls():
         assert torch.isfinite(o_new).all()
         assert rel_err(o_new, o_ref.double().cpu().numpy()) <= tol
         assert rel_err(st_new, st_ref.double().cpu().numpy()) <= tol
+        outs.append(o_new.cpu())
+    # and against the FP64 oracle on one head: both calls are one 2T-token scan
+    head = [5]
+    o_orc, s_orc = oracle_heads(inp, heads=head)
+    assert rel_err(torch.cat(outs, dim=1)[:, :, head], o_orc) <= TOL[torch.bfloat16]
+    assert rel_err(st_new.cpu()[:, head], s_orc) <= TOL[torch.bfloat16]
