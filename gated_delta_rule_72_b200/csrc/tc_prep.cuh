@@ -11,7 +11,8 @@
 //   P_rs = e^{g_r-g_s} (QK^T)_rs, s <= r   (forward)     | readout mask
 //        = e^{g_{r-1}-g_s} (QK^T)_rs, s < r (reverse)    |
 //   T = (I + L)^{-1}                                      (blocked 16x16, CUDA cores)
-//   W = T diag(beta e^g) K,  U = T diag(beta) V           (kind::f16 fp16, single-rounded T)
+//   W = T diag(beta e^g) K,  U = T diag(beta) V           (kind::f16 bf16: T diag(beta e^g)
+//                                                          single, T diag(beta) as a hi/lo pair)
 //   Q~_r = dq_r q_r, dq_r = e^{g_r} (reverse: e^{g_{r-1}});  K~_r = e^{g_63 - g_r} k_r
 //   ds = e^{g_63}
 // and writes them as one fp16 record (tc_common.cuh) with rows in forward
@@ -35,16 +36,17 @@ struct PrepSmem {
     static constexpr int kL = kStage;                 // [64][65] fp32
     static constexpr int kT = kL + 64 * 65 * 4;       // [64][65] fp32
     static constexpr int kX = kT + 64 * 65 * 4;       // 3 x [16][16] fp32
-    static constexpr int kT1 = (kX + 3 * 256 * 4 + 1023) / 1024 * 1024;   // fp16 K-major 64 x 64
-    static constexpr int kT2 = kT1 + 8192;
-    static constexpr int kGate = kT2 + 8192;          // g, beta, dq, dkk, beta e^g
-    static constexpr int kMisc = kGate + 5 * 256;     // key-norm partials [2], record gate [4]
-    static constexpr int kBar = kMisc + 32;           // tma, mma, gram
+    static constexpr int kT1 = (kX + 3 * 256 * 4 + 1023) / 1024 * 1024;   // bf16 K-major 64 x 64
+    static constexpr int kT2h = kT1 + 8192;           // T diag(beta), bf16 hi
+    static constexpr int kT2l = kT2h + 8192;          // and lo
+    static constexpr int kGate = kT2l + 8192;         // g, beta, dq, dkk, beta e^g
+    static constexpr int kMisc = kGate + 5 * 256;     // key-norm partials [2], record gate [4], task [2][4]
+    static constexpr int kBar = kMisc + 64;           // tma, mma, gram
     static constexpr int kCtl = kBar + 32;            // tmem base, abort, ds
     static constexpr int kBytes = kCtl + 16;
     static constexpr int kAlloc = kBytes + 1024;
     static_assert(kStage % 1024 == 0 && kT1 % 1024 == 0, "swizzled areas stay 1024-aligned");
-    // record staging: P and W images over T1 | T2, U over L | T
+    // record staging: P and W images over T1 | T2h, U over L
     static_assert(64 * DV * 2 <= 2 * 64 * 65 * 4, "record staging areas");
     static_assert(kAlloc <= 232448 / 2 - 1024, "two pipelines per SM");
 };
@@ -136,9 +138,19 @@ __device__ __forceinline__ void prep_pipeline(
         while (t < ntasks && !prep_task(po, t, nbh, ndir, nC, dir, c, bh)) t += task_stride;
         return t;
     };
-    auto issue_tma = [&](int t) {
-        int dir, c, bh;
-        prep_task(po, t, nbh, ndir, nC, dir, c, bh);
+    // Task descriptors, decoded once by thread 0 and read by every thread:
+    // two slots (current, next) of {valid, dir, chunk, b*H+h}.
+    int *desc = reinterpret_cast<int *>(smem + SM::kMisc + 32);
+    auto put_desc = [&](int slot, int t) {
+        int dir = 0, c = 0, bh = 0;
+        const bool ok = t < ntasks && prep_task(po, t, nbh, ndir, nC, dir, c, bh);
+        desc[slot * 4 + 0] = ok ? 1 : 0;
+        desc[slot * 4 + 1] = dir;
+        desc[slot * 4 + 2] = c;
+        desc[slot * 4 + 3] = bh;
+    };
+    auto issue_tma = [&](int dir, int c, int bh) {
+        (void)dir;
         const int b = bh / H, h = bh % H, t0 = c * 64;
         unsigned char *st = smem;
         mbar_arrive_expect_tx(tma_bar, SM::kStage);
@@ -159,9 +171,7 @@ __device__ __forceinline__ void prep_pipeline(
     // gates of a task, processing order: thread r < 64 loads row r (raw alpha:
     // the logarithm is taken when the value is used, so the load's latency is
     // not waited for here)
-    auto load_gates = [&](int t, float &al, float &bt) {
-        int dir, c, bh;
-        prep_task(po, t, nbh, ndir, nC, dir, c, bh);
+    auto load_gates = [&](int dir, int c, int bh, float &al, float &bt) {
         const int b = bh / H, h = bh % H;
         const int tok = token_of_row(c, tid, dir);
         const size_t off = ((size_t)b * T + tok) * H + h;
@@ -169,27 +179,57 @@ __device__ __forceinline__ void prep_pipeline(
         bt = tok < T ? beta[off] : 0.f;
     };
 
-    int t = next_valid(first_task);
-    if (t < ntasks && tid == 0) issue_tma(t);
+    int t = 0;   // thread 0: index of the current task
+    if (tid == 0) {
+        t = next_valid(first_task);
+        put_desc(0, t);
+        if (desc[0]) issue_tma(desc[1], desc[2], desc[3]);
+    }
+    // the blocks of T above the block diagonal are zero for every task (nothing
+    // writes them), so they are cleared once
+    for (int e = tid; e < 64 * 64; e += kPrepThreads) {
+        const int i = e >> 6, jj = e & 63;
+        if ((jj >> 4) > (i >> 4)) Tsm[i * 65 + jj] = 0.f;
+    }
+    psync();
     float al_n = 1.f, bt_n = 0.f;
-    if (t < ntasks && tid < 64) load_gates(t, al_n, bt_n);
+    if (tid < 64 && desc[0]) load_gates(desc[1], desc[2], desc[3], al_n, bt_n);
     uint32_t tma_phase = 0, mma_phase = 0, g_phase = 0;
     unsigned int *pending_flag = nullptr;   // thread 0: ready flag of the last record stored
     const uint32_t st_addr = sbase;
+    int slot = 0;
 
-    while (t < ntasks) {
-        int dir, c, bh;
-        prep_task(po, t, nbh, ndir, nC, dir, c, bh);
+    for (;;) {
+        if (!desc[slot * 4]) break;
+        const int dir = desc[slot * 4 + 1], c = desc[slot * 4 + 2], bh = desc[slot * 4 + 3];
+        const int nxt = slot ^ 1;
         const bool rev = dir != 0;
         unsigned char *rec = recs + ((size_t)(dir * nbh + bh) * nC + c) * RC::kStride;
-        const int tn = next_valid(t + task_stride);
+        int tn = 0;
+        if (tid == 0) {
+            tn = next_valid(t + task_stride);
+            put_desc(nxt, tn);
+        }
 
         if (tid < 64) { g_s[tid] = __logf(al_n); beta_s[tid] = bt_n; }
         wait_all(tma_bar, tma_phase);
         tma_phase ^= 1;
         psync();
         if (*abort_s) break;
-        if (tn < ntasks && tid < 64) load_gates(tn, al_n, bt_n);   // next task's gates travel meanwhile
+        // ---- [K; Q] K^T, the two K halves from two issuing threads (it depends on
+        //      the tiles only, so it runs while the gates are prepared) ---------------
+        if (tid == 0 || tid == 64) {
+            const int part = tid >> 6;
+            tc_fence_after();
+            constexpr uint32_t id = idesc(128, 64, 1, 0, 0);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t a = st_addr + part * 16384 + k * 32;
+                mma_bf16(tmem + (part ? kPrepColG2 : kPrepColG), sdesc_sw128(a), sdesc_sw128(a), id, k > 0);
+            }
+            mma_commit(g_bar);
+        }
+        if (tid < 64 && desc[nxt * 4]) load_gates(desc[nxt * 4 + 1], desc[nxt * 4 + 2], desc[nxt * 4 + 3], al_n, bt_n);
         if (warp == 0) {  // inclusive prefix sum of log alpha, 2 rows per lane
             const float a0 = g_s[2 * lane], a1 = g_s[2 * lane + 1];
             float s = a0 + a1;
@@ -228,18 +268,6 @@ __device__ __forceinline__ void prep_pipeline(
                 for (int k = 0; k < 4; ++k) fast = fast && (g_s[16 * k] - g_s[16 * k + 15] < 80.f);
                 reinterpret_cast<int *>(Xsm)[576] = fast ? 1 : 0;
             }
-        }
-        // ---- [K; Q] K^T, the two K halves from two issuing threads ----------------
-        if (tid == 0 || tid == 32) {
-            const int part = tid >> 5;
-            tc_fence_after();
-            constexpr uint32_t id = idesc(128, 64, 1, 0, 0);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t a = st_addr + part * 16384 + k * 32;
-                mma_bf16(tmem + (part ? kPrepColG2 : kPrepColG), sdesc_sw128(a), sdesc_sw128(a), id, k > 0);
-            }
-            mma_commit(g_bar);
         }
         // the previous task's record stores must have read the staging areas; when
         // a chain runs alongside, wait for them to land and flag that record
@@ -329,8 +357,7 @@ __device__ __forceinline__ void prep_pipeline(
             rgate_s[1] = rgate_s[2] = rgate_s[3] = 0.f;
         }
         // ---- T = (I + L)^{-1}, blocked 16 x 16 (processing order); meanwhile the
-        //      other threads turn the tiles into fp16: K and V in place (operands of
-        //      W and U), Q~ and K~ straight into the record -----------------------
+        //      other threads write the record's Q~ and K~ (fp16) from the tiles -------
         if (tid < 64) {
             const int blk = tid >> 4, j = tid & 15, o0 = blk * 16;
             float x[16];
@@ -344,85 +371,117 @@ __device__ __forceinline__ void prep_pipeline(
 #pragma unroll
             for (int i = 0; i < 16; ++i) Tsm[(o0 + i) * 65 + o0 + j] = x[i];
         } else {
-            for (int e = tid - 64; e < 64 * 64; e += kPrepThreads - 64) {
-                const int i = e >> 6, jj = e & 63;
-                if ((jj >> 4) > (i >> 4)) Tsm[i * 65 + jj] = 0.f;
-            }
-            // 16-byte chunks: K blocks (2 x 512), Q blocks (2 x 512), V blocks (DV/64 x 512)
-            constexpr int kChunks = 2048 + (DV / 64) * 512;
-            for (int i = tid - 64; i < kChunks; i += kPrepThreads - 64) {
+            // 16-byte chunks of the record: K~ (2 blocks x 512), Q~ (2 blocks x 512)
+            for (int i = tid - 64; i < 2048; i += kPrepThreads - 64) {
                 const int blk = i >> 9, within = (i & 511) * 16, f = (i & 511) >> 3;
                 const int rr = rev ? 63 - f : f;
-                unsigned char *src;
-                if (blk < 2) src = smem + blk * 16384 + within;                    // K
-                else if (blk < 4) src = smem + (blk - 2) * 16384 + 8192 + within;  // Q
-                else src = smem + SM::kKQ + (blk - 4) * 8192 + within;            // V
+                const bool is_k = blk < 2;
+                const unsigned char *src = smem + (blk & 1) * 16384 + (is_k ? 0 : 8192) + within;
                 const uint4 raw = *reinterpret_cast<const uint4 *>(src);
                 const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
-                uint32_t o16[4], sc16[4];
-                const float scale = blk < 2 ? dkk_s[rr] : dq_s[rr];
+                const float scale = is_k ? dkk_s[rr] : dq_s[rr];
+                uint32_t o16[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 x2 = unpack_bf16(in[e]);
-                    o16[e] = pack_f16(x2.x, x2.y);
-                    sc16[e] = pack_f16(scale * x2.x, scale * x2.y);
+                    o16[e] = pack_f16(scale * x2.x, scale * x2.y);
                 }
-                if (blk < 2) {
-                    *reinterpret_cast<uint4 *>(src) = make_uint4(o16[0], o16[1], o16[2], o16[3]);
-                    *reinterpret_cast<uint4 *>(rec + RC::kK + blk * 8192 + within) =
-                        make_uint4(sc16[0], sc16[1], sc16[2], sc16[3]);
-                } else if (blk < 4) {
-                    *reinterpret_cast<uint4 *>(rec + RC::kQW + (blk - 2) * 16384 + within) =
-                        make_uint4(sc16[0], sc16[1], sc16[2], sc16[3]);
-                } else {
-                    *reinterpret_cast<uint4 *>(src) = make_uint4(o16[0], o16[1], o16[2], o16[3]);
-                }
+                unsigned char *dst = rec + (is_k ? RC::kK + (blk & 1) * 8192 : RC::kQW + (blk & 1) * 16384) + within;
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(o16[0], o16[1], o16[2], o16[3]);
             }
             __threadfence();   // the record's Q~ and K~ are published with its flag
         }
         psync();
-        // off-diagonal blocks by bands: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj, i = j + band,
-        // each thread a 2 x 2 tile (independent accumulators, conflict-free loads)
-        for (int band = 1; band < 4; ++band) {
-            const int nblk = 4 - band;
-            for (int e = tid; e < nblk * 64; e += kPrepThreads) {
-                const int j = e >> 6, ti = (e >> 3) & 7, tj = e & 7;
-                const int i = j + band;
-                const int a = i * 16 + 2 * ti, bc = j * 16 + 2 * tj;
-                float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
-                for (int m = j * 16; m < i * 16; ++m) {
+        // off-diagonal blocks by recursive doubling (processing order):
+        //   level 2, within each 32-block b: T_10 = -T_11 (L_10 T_00)   (16 x 16 blocks)
+        //   level 3: T_[32:64, 0:32] = -T_[32:64, 32:64] (L_[32:64, 0:32] T_[0:32, 0:32])
+        // T is stored lower-triangular with explicit zeros above the diagonal, so
+        // the sums run over whole blocks (unrolled); each thread owns a 2 x 2 tile.
+        if (tid < 128) {   // level 2, X = L_10 T_00 into Xsm[b][16][16]
+            const int b2 = tid >> 6, ti = (tid >> 3) & 7, tj = tid & 7, base = 32 * b2;
+            const int a = base + 16 + 2 * ti, bc = base + 2 * tj;
+            float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float l0 = Lsm[a * 65 + base + m], l1 = Lsm[(a + 1) * 65 + base + m];
+                const float t0 = Tsm[(base + m) * 65 + bc], t1 = Tsm[(base + m) * 65 + bc + 1];
+                x00 = fmaf(l0, t0, x00); x01 = fmaf(l0, t1, x01);
+                x10 = fmaf(l1, t0, x10); x11 = fmaf(l1, t1, x11);
+            }
+            float *xb = Xsm + b2 * 256 + (2 * ti) * 16 + 2 * tj;
+            xb[0] = x00; xb[1] = x01; xb[16] = x10; xb[17] = x11;
+        }
+        psync();
+        if (tid < 128) {   // level 2, T_10 = -T_11 X
+            const int b2 = tid >> 6, ti = (tid >> 3) & 7, tj = tid & 7, base = 32 * b2;
+            const int a = base + 16 + 2 * ti, bc = base + 2 * tj;
+            const float *xb = Xsm + b2 * 256 + 2 * tj;
+            float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float t0 = Tsm[a * 65 + base + 16 + m], t1 = Tsm[(a + 1) * 65 + base + 16 + m];
+                const float x0 = xb[m * 16], x1 = xb[m * 16 + 1];
+                y00 = fmaf(t0, x0, y00); y01 = fmaf(t0, x1, y01);
+                y10 = fmaf(t1, x0, y10); y11 = fmaf(t1, x1, y11);
+            }
+            Tsm[a * 65 + bc] = -y00; Tsm[a * 65 + bc + 1] = -y01;
+            Tsm[(a + 1) * 65 + bc] = -y10; Tsm[(a + 1) * 65 + bc + 1] = -y11;
+        }
+        psync();
+        // level 3, X = L_[32:64, 0:32] T_[0:32, 0:32] (32 x 32, fp32, stride 33) in the
+        // T2 image area (free until the T images).  Thread tile rows 2*(tid & 15),
+        // columns 2*(tid >> 4): a warp's columns are 4w .. 4w+3, so the rows of T
+        // above 4w (zero) are skipped by whole 8-row steps.
+        float *X3 = reinterpret_cast<float *>(smem + SM::kT2h);
+        {
+            const int ti = tid & 15, tj = tid >> 4;
+            const int a = 32 + 2 * ti, bc = 2 * tj;
+            const int m0 = (warp * 4) & ~7;
+            float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) {
+                if (c8 * 8 + 8 <= m0) continue;    // warp-uniform
+#pragma unroll
+                for (int mm = 0; mm < 8; ++mm) {
+                    const int m = c8 * 8 + mm;
                     const float l0 = Lsm[a * 65 + m], l1 = Lsm[(a + 1) * 65 + m];
                     const float t0 = Tsm[m * 65 + bc], t1 = Tsm[m * 65 + bc + 1];
                     x00 = fmaf(l0, t0, x00); x01 = fmaf(l0, t1, x01);
                     x10 = fmaf(l1, t0, x10); x11 = fmaf(l1, t1, x11);
                 }
-                float *xb = Xsm + j * 256 + (2 * ti) * 16 + 2 * tj;
-                xb[0] = x00; xb[1] = x01; xb[16] = x10; xb[17] = x11;
             }
-            psync();
-            for (int e = tid; e < nblk * 64; e += kPrepThreads) {
-                const int j = e >> 6, ti = (e >> 3) & 7, tj = e & 7;
-                const int i = j + band;
-                const int a = i * 16 + 2 * ti, bc = j * 16 + 2 * tj;
-                const float *xb = Xsm + j * 256 + 2 * tj;
-                float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+            float *xb = X3 + (2 * ti) * 33 + bc;
+            xb[0] = x00; xb[1] = x01; xb[33] = x10; xb[34] = x11;
+        }
+        psync();
+        {   // level 3, T_[32:64, 0:32] = -T_[32:64, 32:64] X: tile rows 2*(tid >> 4) (a
+            // warp's rows 4w .. 4w+3, so T's zero columns past them are skipped),
+            // columns 2*(tid & 15)
+            const int ti = tid >> 4, tj = tid & 15;
+            const int a = 32 + 2 * ti, bc = 2 * tj;
+            const int m1 = warp * 4 + 4;          // T_[a, 32+m] = 0 for m >= m1
+            float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float t0 = Tsm[a * 65 + i * 16 + m], t1 = Tsm[(a + 1) * 65 + i * 16 + m];
-                    const float x0 = xb[m * 16], x1 = xb[m * 16 + 1];
+            for (int c8 = 0; c8 < 4; ++c8) {
+                if (c8 * 8 >= m1) continue;        // warp-uniform
+#pragma unroll
+                for (int mm = 0; mm < 8; ++mm) {
+                    const int m = c8 * 8 + mm;
+                    const float t0 = Tsm[a * 65 + 32 + m], t1 = Tsm[(a + 1) * 65 + 32 + m];
+                    const float x0 = X3[m * 33 + bc], x1 = X3[m * 33 + bc + 1];
                     y00 = fmaf(t0, x0, y00); y01 = fmaf(t0, x1, y01);
                     y10 = fmaf(t1, x0, y10); y11 = fmaf(t1, x1, y11);
                 }
-                Tsm[a * 65 + bc] = -y00; Tsm[a * 65 + bc + 1] = -y01;
-                Tsm[(a + 1) * 65 + bc] = -y10; Tsm[(a + 1) * 65 + bc + 1] = -y11;
             }
-            psync();
+            Tsm[a * 65 + bc] = -y00; Tsm[a * 65 + bc + 1] = -y01;
+            Tsm[(a + 1) * 65 + bc] = -y10; Tsm[(a + 1) * 65 + bc + 1] = -y11;
         }
+        psync();
         // the P store has read its staging area (the T images go there next)
         if (tid == 0) bulk_wait_read_all();
         psync();
-        // ---- A operands T diag(beta e^g) and T diag(beta) (fp16), in forward
-        //      row/column order (mirrored for the reverse direction) ------------------
+        // ---- A operands T diag(beta e^g) (bf16) and T diag(beta) (bf16 hi/lo pair),
+        //      in forward row/column order (mirrored for the reverse direction) -------
         for (int cell = tid; cell < 64 * 8; cell += kPrepThreads) {
             const int fr = cell & 63, fc0 = (cell >> 6) * 8;
             const int r = rev ? 63 - fr : fr;
@@ -434,28 +493,30 @@ __device__ __forceinline__ void prep_pipeline(
                 a[e] = tv * bg_s[s];
                 bvals[e] = tv * beta_s[s];
             }
-            uint4 h1, h2;
-            h1.x = pack_f16(a[0], a[1]); h1.y = pack_f16(a[2], a[3]);
-            h1.z = pack_f16(a[4], a[5]); h1.w = pack_f16(a[6], a[7]);
-            h2.x = pack_f16(bvals[0], bvals[1]); h2.y = pack_f16(bvals[2], bvals[3]);
-            h2.z = pack_f16(bvals[4], bvals[5]); h2.w = pack_f16(bvals[6], bvals[7]);
+            uint4 h1, h2, l2;
+            h1.x = pack_bf16(a[0], a[1]); h1.y = pack_bf16(a[2], a[3]);
+            h1.z = pack_bf16(a[4], a[5]); h1.w = pack_bf16(a[6], a[7]);
+            split2(bvals[0], bvals[1], h2.x, l2.x); split2(bvals[2], bvals[3], h2.y, l2.y);
+            split2(bvals[4], bvals[5], h2.z, l2.z); split2(bvals[6], bvals[7], h2.w, l2.w);
             const int off = kmaj64(fr, fc0);
             *reinterpret_cast<uint4 *>(smem + SM::kT1 + off) = h1;
-            *reinterpret_cast<uint4 *>(smem + SM::kT2 + off) = h2;
+            *reinterpret_cast<uint4 *>(smem + SM::kT2h + off) = h2;
+            *reinterpret_cast<uint4 *>(smem + SM::kT2l + off) = l2;
         }
         fence_async_shared();
         psync();
-        // ---- W = T1 K and U = T2 V on the tensor cores (fp16 K and V in the tiles)
+        // ---- W = T1 K and U = T2 V on the tensor cores (K and V straight from the tiles)
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t idw = idesc(64, 128, 0, 0, 1);
-            constexpr uint32_t idu = idesc(64, DV, 0, 0, 1);
+            constexpr uint32_t idw = idesc(64, 128, 1, 0, 1);
+            constexpr uint32_t idu = idesc(64, DV, 1, 0, 1);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
                 mma_bf16(tmem + kPrepColW, sdesc_noswz(sbase + SM::kT1 + 2 * s * 1024, 1024, 128),
                          sdesc_sw128_mn(st_addr + s * 2048, 16384), idw, s > 0);
-                mma_bf16(tmem + kPrepColU, sdesc_noswz(sbase + SM::kT2 + 2 * s * 1024, 1024, 128),
-                         sdesc_sw128_mn(st_addr + SM::kKQ + s * 2048, 8192), idu, s > 0);
+                const uint64_t bv = sdesc_sw128_mn(st_addr + SM::kKQ + s * 2048, 8192);
+                mma_bf16(tmem + kPrepColU, sdesc_noswz(sbase + SM::kT2h + 2 * s * 1024, 1024, 128), bv, idu, s > 0);
+                mma_bf16(tmem + kPrepColU, sdesc_noswz(sbase + SM::kT2l + 2 * s * 1024, 1024, 128), bv, idu, 1);
             }
             mma_commit(mma_bar);
         }
@@ -463,7 +524,7 @@ __device__ __forceinline__ void prep_pipeline(
         mma_phase ^= 1;
         tc_fence_after();
         // the tiles are consumed: fetch the next task's while this one is written out
-        if (tn < ntasks && tid == 0) issue_tma(tn);
+        if (tid == 0 && desc[nxt * 4]) issue_tma(desc[nxt * 4 + 1], desc[nxt * 4 + 2], desc[nxt * 4 + 3]);
         // ---- record: W image and U rows (fp16), staged in the areas the products
         //      are done with (T images, L/T) and written by bulk stores ---------------
         {
@@ -512,7 +573,8 @@ __device__ __forceinline__ void prep_pipeline(
             bulk_store(rec + RC::kGate, rgate_s, 16);
             bulk_commit_group();
         }
-        t = tn;
+        if (tid == 0) t = tn;
+        slot = nxt;
     }
 
     if (tid == 0) {
