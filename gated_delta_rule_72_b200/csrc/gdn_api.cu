@@ -201,13 +201,8 @@ size_t tc_record_bytes(int dv) {
 }
 
 // Tensor-core path workspace: one record per chunk, head and direction, one
-// ready flag and one log bound per record; then, bidirectional only, the fp32
-// sum buffer of the two directions (bf16 o; an fp32 o is its own sum) and one
-// counter per output tile.
-size_t tc_pair_counters(int B, int T, int H) {
-    const size_t nC = (size_t)(T + kChunk - 1) / kChunk;
-    return (size_t)B * H * nC;   // one per (b, h, chunk) output tile
-}
+// ready flag and one log bound per record; then, bidirectional with a bf16
+// o only, the fp32 sum of the two directions (an fp32 o is its own sum).
 
 size_t plan_workspace(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dtype o_dt, int bidir) {
     if (T == 0) return 0;
@@ -217,10 +212,7 @@ size_t plan_workspace(int B, int T, int H, int dk, int dv, gdn_dtype dt, gdn_dty
         size_t bytes = round_up(nrec * tc_record_bytes(dv), 256);
         bytes += round_up(nrec * sizeof(unsigned int), 256);   // ready flags
         bytes += round_up(nrec * sizeof(float), 256);          // log bounds of the chunk maps
-        if (bidir) {
-            if (o_dt == GDN_BF16) bytes += round_up((size_t)B * T * H * dv * sizeof(float), 256);
-            bytes += round_up(tc_pair_counters(B, T, H) * sizeof(unsigned int), 256);
-        }
+        if (bidir && o_dt == GDN_BF16) bytes += round_up((size_t)B * T * H * dv * sizeof(float), 256);
         return bytes;
     }
     return simt_workspace(B, T, H, dk, dv, bidir);
@@ -285,15 +277,10 @@ int sm_count() {
     return n;
 }
 
-// Output tile map: fp32 boxes of 32 columns, bf16 boxes of 64 (128-byte rows,
-// 128B swizzle, as the chain stages them).
-bool encode_out_map(CUtensorMap *m, const void *target, const Args &a, int dv, bool f32) {
-    return encode_map(m, target, a.B, a.T, a.H, dv, f32 ? 32 : 64, 128, f32 ? 4 : 2);
-}
-
 // Segmentation of the chunk walks and the split of the SMs.
 //   G segments of L chunks per chain; fused: n_chain chain CTAs beside
-//   n_prep CTAs of two prep pipelines (one cooperative launch).
+//   n_prep CTAs of two prep pipelines (one cooperative launch); else prep on
+//   every SM, then the chains.
 struct TcPlan {
     bool fused;
     int G, L, n_chain, n_prep;
@@ -306,41 +293,49 @@ std::atomic<int> g_chain_segments{-1};
 // Fewest prep CTAs (two pipelines each) worth a fused launch: below this the
 // prep would lag the chains and two launches do better.
 constexpr int kMinFusedPrepCtas = 32;
-// Share of the SMs given to chain CTAs in a fused launch, in 1/16ths.
-constexpr int kChainShare16 = 6;
 // Fewest chunks per segment (a segment also walks back a few chunks first).
 constexpr int kMinSegChunks = 16;
 // Tail positions of every segment the prep produces first (the next
 // segment's walk back reads them before anything else).
 constexpr int kTailFirst = 12;
 
+// Automatic plan (from B200 timings of the d = 128 workloads): when the walks
+// are long enough to cut, prep on every SM and then one wave of chain CTAs
+// (G = SMs / chains, at least 16 chunks per segment: a 32k-token causal scan
+// of 12 heads 0.39 ms against 0.49 ms fused with 4 segments; bidirectional
+// 75k tokens of 20 heads 3.0 ms against 4.2 ms fused); when they are not
+// (short calls), one fused launch whose prep runs beside the chains so the
+// first chunk's record is ready early.  A forced segment count takes the
+// fused launch where the SMs allow it.
 TcPlan plan_tc(int chains, int nC, bool coop) {
     const int sms = sm_count();
     TcPlan p{};
-    p.fused = coop && chains + kMinFusedPrepCtas <= sms;
-    int G;
     const int forced = g_chain_segments.load(std::memory_order_relaxed);
     const int gmax = nC / kMinSegChunks > 1 ? nC / kMinSegChunks : 1;
+    int G;
     if (forced > 0) {
-        G = forced;
-    } else if (p.fused) {
-        G = (sms * kChainShare16 / 16) / chains;
-        if (G > gmax) G = gmax;
+        G = forced < nC ? forced : nC;
+        p.fused = coop && (long long)chains * G + kMinFusedPrepCtas <= sms;
     } else {
         G = sms / chains;
         if (G > gmax) G = gmax;
+        if (G < 1) G = 1;
+        p.fused = G == 1 && coop && chains + kMinFusedPrepCtas <= sms;
     }
-    if (G < 1) G = 1;
-    if (G > nC) G = nC;
     p.L = (nC + G - 1) / G;
     p.G = (nC + p.L - 1) / p.L;
     p.n_chain = chains * p.G;
-    if (p.fused && p.n_chain + kMinFusedPrepCtas > sms) p.fused = false;
     p.n_prep = p.fused ? sms - p.n_chain : 0;
     p.po.G = p.G;
     p.po.L = p.L;
     p.po.tail = p.G > 1 ? (p.L < kTailFirst ? p.L : kTailFirst) : 0;
     return p;
+}
+
+// Output tile map: fp32 boxes of 32 columns, bf16 boxes of 64 (128-byte rows,
+// 128B swizzle, as the chain stages them).
+bool encode_out_map(CUtensorMap *m, const void *target, const Args &a, int dv, bool f32) {
+    return encode_map(m, target, a.B, a.T, a.H, dv, f32 ? 32 : 64, 128, f32 ? 4 : 2);
 }
 
 template <int DV>
@@ -381,8 +376,8 @@ gdn_status launch_chain(const Args &a, const CUtensorMap &mo, const unsigned cha
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kAlloc) != cudaSuccess)
         return GDN_ERR_CUDA;
     gdn::LaunchScope ls(ndir == 2 ? "tc_chain_bidir" : "tc_chain", a.stream);
-    kern<<<dim3(seg.G, a.B * a.H, ndir), gdn::tc2::kChainThreads, SM::kAlloc, a.stream>>>(mo, recs, states, out, seg,
-                                                                                          a.H, nC, err);
+    kern<<<dim3(seg.G, a.B * a.H, ndir), gdn::tc2::kChainThreads, SM::kAlloc, a.stream>>>(mo, recs, states, out,
+                                                                                          seg, a.H, nC, err);
     return launch_status();
 }
 
@@ -453,16 +448,13 @@ gdn_status run_tc(const Args &a, int bidir) {
     const size_t n = (size_t)a.B * a.T * a.H * DV;
     if (bidir) {
         // both directions in one launch, adding up in fp32 (in o itself for an
-        // fp32 o, else in a buffer that is then rounded into o)
+        // fp32 o, else in a buffer that is then rounded into o), from zero
         if (!f32_out) {
             target = p;
             p += round_up(n * sizeof(float), 256);
         }
         out.mode = gdn::tc2::kOutPair;
-        out.cnt = reinterpret_cast<unsigned int *>(p);
-        if (cudaMemsetAsync(out.cnt, 0, tc_pair_counters(a.B, a.T, a.H) * sizeof(unsigned int), a.stream) !=
-            cudaSuccess)
-            return GDN_ERR_CUDA;
+        if (cudaMemsetAsync(target, 0, n * sizeof(float), a.stream) != cudaSuccess) return GDN_ERR_CUDA;
     } else {
         out.mode = gdn::tc2::kOutStore;
     }

@@ -8,29 +8,35 @@
 //   [Y; X] = [Q~; W] S                  one M=128 product, two K halves
 //   Delta  = U - X                      (fp16 D)
 //   S     <- ds S + K~^T D
-//   O      = Y + P D                    P D accumulates onto Y in TMEM
+//   O      = Y + P D
 // with Q~ = diag(e^g) Q and K~ = diag(e^{g_last - g}) K prepared by the prep
 // kernel, so no per-row gate enters the chain.  Stacking Q~ over W makes Y
 // and X one instruction stream: Y lands in TMEM lanes 0-63, X in 64-127.
-// Each product is split over two MMA streams (two issuing threads, two
-// accumulators): a dependent tcgen05 MMA completes about every 130 cycles
-// whatever N is up to 256, so the K halves run side by side.
+// The chain's own products are split over two MMA streams (two issuing
+// threads, two accumulators): a dependent tcgen05 MMA completes about every
+// 130 cycles whatever N is up to 256, so the halves run side by side.
 //
-// TMEM (4 x DV columns): [XA | XB | KA | KB]; XA/XB hold the two K halves of
-// [Y; X] and then, in their lanes 0-63, Y + P D (two token halves of P D);
-// KA/KB the two token halves of K~^T D.
+// TMEM (4 x DV columns): XA, XB hold the two K halves of [Y; X]; KA and then
+// XA (once read) the two token halves of K~^T D; OY holds O: the Y rows copy
+// Y there (tcgen05.st) while the X rows form D, and P D accumulates onto it.
+// So the next chunk's [Q~; W] S waits only for the state, never for the
+// output, and P D stays off the chain's critical path.
 //
 // Roles (20 warps).  The 16 epilogue warps cover the 128 TMEM lanes four
 // times (warp w reads lane quarter w % 4, columns DV/4 * (w / 4) .. +DV/4-1):
 //   quarters 2, 3 (X rows)  Delta = U - X -> D             (critical path)
+//   quarters 0, 1 (Y rows)  Y -> OY, then O = OY -> staged output tile
 //   all                     S <- ds S + K~^T D, thread = one row of S
-//   quarters 0, 1 (Y rows)  O = Y + P D -> staged output tile
-// Warps 16 and 17 issue the two halves of every product, warp 18 loads the
-// records (one bulk copy per chunk, double-buffered) and warp 19 stores the
-// output tiles.  A stage is free again once both issuers' products are done
-// and every epilogue warp has read it (a Y warp's output tile staged there has
-// been read by its store: the storer arrives for the 8 Y warps).  Roles meet on mbarriers; every wait is bounded and a wait
-// that gives up sets an error flag and lets the kernel wind down.
+// Warps 16 and 17 issue the two halves of the chain's products (16 also
+// P D) and warp 18 loads the records (one bulk copy per chunk,
+// double-buffered).  A stage is free again once both issuers' products are
+// done and every epilogue warp has read it.  The Y rows write the output
+// straight to global memory from registers.  Roles meet on mbarriers; every
+// wait is bounded and a wait that gives up sets an error flag and lets the
+// kernel wind down.  A
+// tcgen05.commit covers every earlier MMA of its issuing thread, so the
+// [Y; X] product of a chunk completing also means that thread's P D of the
+// chunk before has completed (and no longer reads D).
 //
 // Sequence parallelism.  A chain of n chunks is cut into G segments of L
 // chunks of the walk; segment g emits the outputs of walk steps
@@ -47,13 +53,9 @@
 // state.  With fast-forgetting gates the walk back is a few chunks; with
 // alpha = 1 it is the whole prefix (correct, but no faster than one segment).
 //
-// Bidirectional mode runs both directions in one launch, and both write the
-// same fp32 output tiles.  An atomic counter per tile decides the order: the
-// first of the two CTAs TMA-stores its tile and then marks it landed; the
-// second waits for that mark (the two directions reach a given tile at very
-// different times, so it seldom waits) and TMA-reduce-adds its own tile onto
-// it.  The first one's mark does not depend on any other CTA, and the second
-// only waits on a CTA that is already running.
+// Bidirectional mode runs both directions in one launch; both add their rows
+// into one zeroed fp32 sum with 16-byte atomic adds (an fp32 add of two values
+// does not depend on their order, so the sum is deterministic).
 #pragma once
 
 #include "tc_common.cuh"
@@ -67,17 +69,21 @@ struct ChainSmem {
     // Two stages, each one record image (Rec<DV>).  The operands the
     // epilogues write are 128B-swizzled MN-major, as a tile load would write
     // them: S (K = d_k = 128 rows per 64-column group) and D (K = 64 tokens).
-    // The output tile is staged over the stage's [Q~; W] area, which the
-    // products are done with by then.
+    // The output tile is staged in its own buffer, so a stage is free for the
+    // next record as soon as its products are done.
     static constexpr int kStage = Rec<DV>::kStage;
     static constexpr int kGrpS = 128 * 128;
     static constexpr int kGrpD = 64 * 128;
     static constexpr int kS = 2 * kStage;
     static constexpr int kD = kS + (DV / 64) * kGrpS;
-    static constexpr int kBar = kD + (DV / 64) * kGrpD;
+    static constexpr int kO = kD + (DV / 64) * kGrpD;    // output tile, fp32 staging
+    static constexpr int kOBytes = 64 * DV * 4;
+    static constexpr int kBar = kO + kOBytes;
     static constexpr int kCtl = kBar + 256;
     static constexpr int kBytes = kCtl + 32;
-    static constexpr int kAlloc = kBytes + 1024;
+    // the dynamic shared memory is declared 1024-aligned (and checked at run
+    // time), so no alignment slack is allocated
+    static constexpr int kAlloc = kBytes;
     static_assert(kStage % 1024 == 0 && kS % 1024 == 0 && kD % 1024 == 0, "swizzled operands stay 1024-aligned");
     static_assert(kAlloc <= 232448, "shared memory budget");
 };
@@ -93,20 +99,14 @@ struct ChainStates {
     float *out[2];
 };
 
-// Output of a chain.  kOutStore: tm_o maps o ([B, T, H, DV], Tout).  kOutPair
-// (both directions): tm_o maps an fp32 [B, T, H, DV] sum (o itself when Tout
-// is float), cnt holds one counter per output tile (b, h, chunk), zero on entry.
+// Output of a chain.  kOutStore: tm_o maps o ([B, T, H, DV], Tout), each
+// tile stored once.  kOutPair (both directions): tm_o maps an fp32
+// [B, T, H, DV] sum (o itself when Tout is float), zero on entry, onto which
+// each direction's tiles are reduce-added by TMA (an fp32 add of two values,
+// so the order does not matter).
 template <typename Tout>
 struct ChainOut {
-    unsigned int *cnt;
     int mode;
-};
-
-// Segmentation of the chunk walk: G segments of L chunks; lb holds the log
-// norm bound of every chunk's state map, [dir][b*H+h][chunk].
-struct ChainSeg {
-    int G, L;
-    const float *lb;
 };
 
 // Staging of one output tile (64 rows x DV columns) for its TMA store: byte
@@ -118,6 +118,13 @@ __device__ __forceinline__ int out_stage_off(int row, int col) {
     if (sizeof(Tout) == 4) return (col >> 5) * 8192 + swz128(row * 128 + (col & 31) * 4);
     return (col >> 6) * 8192 + swz128(row * 128 + (col & 63) * 2);
 }
+
+// Segmentation of the chunk walk: G segments of L chunks; lb holds the log
+// norm bound of every chunk's state map, [dir][b*H+h][chunk].
+struct ChainSeg {
+    int G, L;
+    const float *lb;
+};
 
 // The chain of one (segment, bh, dir): block kChainThreads, `smem` its
 // 1024-aligned shared memory (ChainSmem<DV>), nbh = B * H.  With `ready`
@@ -135,15 +142,15 @@ __device__ __forceinline__ void chain_body(
     constexpr int NC = DV / 4;          // columns per epilogue warp
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kBar);
     uint64_t *full = bars + 0;         // [2] stage loaded                         (loader -> all)
-    uint64_t *free_st = bars + 2;      // [2] stage consumed: A, B, 16 warps   (-> loader)
+    uint64_t *free_st = bars + 2;      // [2] stage consumed: A, B, 16 warps     (-> loader)
     uint64_t *xy_bar = bars + 4;       // [Y; X] complete, 2 commits               (A, B -> X warps)
     uint64_t *d_bar = bars + 5;        // D written, 8 X warps                     (-> A, B)
     uint64_t *s_bar = bars + 6;        // K~^T D complete, 2 commits               (-> epilogue)
     uint64_t *r_bar = bars + 7;        // S rewritten, 16 warps                    (-> A, B)
-    uint64_t *pd_bar = bars + 8;       // Y + P D complete, 2 commits              (-> Y warps)
-    uint64_t *o_read = bars + 9;       // Y + P D read from TMEM, 8 Y warps        (-> A, B)
+    uint64_t *pd_bar = bars + 8;       // Y + P D complete in OY, 1 commit          (-> Y warps)
+    uint64_t *y_bar = bars + 9;        // Y moved to OY (Y lanes of XA, XB free), 8 Y warps (-> A, B)
     uint64_t *o_bar = bars + 10;       // output tile staged, 8 Y warps            (-> storer)
-    uint64_t *o_seen = bars + 11;      // storer has seen o_bar's phase            (-> Y warps)
+    uint64_t *o_free = bars + 11;      // output buffer read by its store          (storer -> Y warps)
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + SM::kCtl);
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + SM::kCtl + 4);
     volatile int *w0_s = reinterpret_cast<volatile int *>(smem + SM::kCtl + 8);
@@ -154,7 +161,7 @@ __device__ __forceinline__ void chain_body(
     const uint32_t sbase = smem_u32(smem);
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int n0 = cg * NC;                                 // this warp's columns
-    constexpr uint32_t kColXA = 0, kColXB = DV, kColKA = 2 * DV, kColKB = 3 * DV;
+    constexpr uint32_t kColXA = 0, kColXB = DV, kColKA = 2 * DV, kColOY = 3 * DV;
     constexpr uint32_t kCols = 4 * DV;
     const unsigned char *rec_base = recs + (size_t)(dir * nbh + bh) * nC * RC::kStride;
     const size_t flag_base = (size_t)(dir * nbh + bh) * nC;
@@ -172,10 +179,10 @@ __device__ __forceinline__ void chain_body(
         mbar_init(d_bar, 8);
         mbar_init(s_bar, 2);
         mbar_init(r_bar, 16);
-        mbar_init(pd_bar, 2);
-        mbar_init(o_read, 8);
+        mbar_init(pd_bar, 1);
+        mbar_init(y_bar, 8);
         mbar_init(o_bar, 8);
-        mbar_init(o_seen, 1);
+        mbar_init(o_free, 1);
         fence_mbar_init();
         *abort_s = 0;
         prefetch_tensormap(tm_o);
@@ -272,19 +279,20 @@ __device__ __forceinline__ void chain_body(
         }
         __syncwarp();
     } else if (warp == 16 || warp == 17) {
-        // ===== issuers A (warp 16) and B (warp 17): one half of every product
+        // ===== issuers A (warp 16) and B (warp 17): one half of each chain product;
+        // A also P D onto OY
         if (lane == 0) {
             const int part = warp - 16;
             const uint32_t colX = part ? kColXB : kColXA;
-            const uint32_t colK = part ? kColKB : kColKA;
-            uint32_t full_phases = 0, d_phase = 0, r_phase = 0, or_phase = 0;
+            const uint32_t colK = part ? kColXA : kColKA;   // B's half of K~^T D reuses XA
+            uint32_t full_phases = 0, d_phase = 0, r_phase = 0, y_phase = 0;
             for (int step = 0; step < nsteps; ++step) {
                 const int buf = step & 1;
                 const uint32_t st = sbase + buf * SM::kStage;
                 wait_on(&full[buf], (full_phases >> buf) & 1u);
                 full_phases ^= 1u << buf;
+                // S rewritten (and K~^T D read out of KA and XA)
                 if (step > 0) { wait_on(r_bar, r_phase); r_phase ^= 1; }
-                if (step > out0) { wait_on(o_read, or_phase); or_phase ^= 1; }   // Y + P D drained
                 if (*abort_s) break;
                 tc_fence_after();
                 // [Y; X] half: d_k rows 64*part .. +63 of S
@@ -294,8 +302,11 @@ __device__ __forceinline__ void chain_body(
                     mma_bf16(tmem + colX, a, adv(dS, (part * 4 + k) * 2048), idXY, k > 0);
                 }
                 mma_commit(xy_bar);
+                // D written (X rows read) and Y moved to OY (Y rows read)
                 wait_on(d_bar, d_phase);
                 d_phase ^= 1;
+                wait_on(y_bar, y_phase);
+                y_phase ^= 1;
                 if (*abort_s) break;
                 tc_fence_after();
                 // K~^T D half: tokens 32*part .. +31
@@ -306,14 +317,12 @@ __device__ __forceinline__ void chain_body(
                     mma_bf16(tmem + colK, adv(dK, s * 2048), adv(dD, s * 2048), idKD, k > 0);
                 }
                 mma_commit(s_bar);
-                if (step >= out0) {
-                    // P D half (source tokens 32*part .. +31), onto Y.  M = 128: rows
-                    // 64-127 of A run on into U (finite; their lanes hold X, already read)
+                if (part == 0 && step >= out0) {
+                    // P D onto Y in OY.  M = 128: rows 64-127 of A run on into U (finite;
+                    // their lanes of OY are never read)
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const int s = part * 2 + k;
-                        mma_bf16(tmem + colX, sdesc_sw128(st + RC::kP + s * 32), adv(dD, s * 2048), idXY, 1);
-                    }
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(tmem + kColOY, sdesc_sw128(st + RC::kP + k * 32), adv(dD, k * 2048), idXY, 1);
                     mma_commit(pd_bar);
                 }
                 mma_commit(&free_st[buf]);
@@ -321,37 +330,21 @@ __device__ __forceinline__ void chain_body(
         }
         __syncwarp();
     } else if (warp == 19) {
-        // ===== storer: the staged output tile leaves by TMA; in a bidirectional
-        // scan the second of the two directions adds its tile onto the first's
+        // ===== storer: the staged output tile leaves by TMA (a bidirectional scan
+        // reduce-adds both directions' tiles onto the zeroed fp32 sum)
         if (lane == 0) {
+            const bool f32t = sizeof(Tout) == 4 || out.mode == kOutPair;
+            const unsigned char *ob = smem + SM::kO;
             uint32_t o_phase = 0;
             for (int step = out0; step < nsteps; ++step) {
-                const int buf = step & 1;
                 const int c = chunk_of(w0 + step);
                 wait_on(o_bar, o_phase);
                 o_phase ^= 1;
-                mbar_arrive(o_seen);   // o_bar may complete its next phase
                 if (*abort_s) break;
-                const unsigned char *ob = smem + buf * SM::kStage + RC::kQW;
-                bool add = false;      // TMA-reduce-add onto the other direction's tile
-                size_t tile = 0;
-                if (out.mode == kOutPair) {
-                    tile = (size_t)bh * nC + c;
-                    if (atomicAdd(out.cnt + tile, 1u) != 0u) {
-                        // second: wait for the first one's "landed" mark (+2)
-                        if (!spin_until_geq(out.cnt + tile, 3u, kFlagWaitNs)) {
-                            *abort_s = 1;
-                            if (err) atomicAdd(err, 1u);
-                            break;
-                        }
-                        fence_proxy_async_global();
-                        add = true;
-                    }
-                }
-                if (sizeof(Tout) == 4 || out.mode == kOutPair) {
+                if (f32t) {
 #pragma unroll
                     for (int x = 0; x < DV / 32; ++x) {
-                        if (add) tma_reduce_add_4d(tm_o, ob + x * 8192, 32 * x, h, c * 64, b);
+                        if (out.mode == kOutPair) tma_reduce_add_4d(tm_o, ob + x * 8192, 32 * x, h, c * 64, b);
                         else tma_store_4d(tm_o, ob + x * 8192, 32 * x, h, c * 64, b);
                     }
                 } else {
@@ -359,14 +352,8 @@ __device__ __forceinline__ void chain_body(
                     for (int x = 0; x < DV / 64; ++x) tma_store_4d(tm_o, ob + x * 8192, 64 * x, h, c * 64, b);
                 }
                 bulk_commit_group();
-                bulk_wait_read_all();            // the staging area may be reused after this
-                mbar_arrive_cnt(&free_st[buf], 8);   // on behalf of the 8 Y warps
-                if (out.mode == kOutPair && !add) {
-                    bulk_wait_all();             // landed in global memory: mark it (+2)
-                    fence_proxy_async_global();
-                    __threadfence();
-                    atomicAdd(out.cnt + tile, 2u);
-                }
+                bulk_wait_read_all();            // the buffer may be refilled after this
+                mbar_arrive(o_free);
             }
             bulk_wait_all();   // the output stores have landed
         }
@@ -375,19 +362,25 @@ __device__ __forceinline__ void chain_body(
         // ============================ epilogue warps (0..15) ========================
         const bool xrows = quarter >= 2;                 // TMEM lanes 64-127 hold X
         const int r = xrows ? d_row - 64 : d_row;        // token row (forward order) of this lane
-        uint32_t full_phases = 0, xy_phase = 0, s_phase = 0, pd_phase = 0, os_phase = 0;
+        uint32_t full_phases = 0, xy_phase = 0, s_phase = 0, pd_phase = 0;
         for (int step = 0; step < nsteps; ++step) {
             const int buf = step & 1;
+            const bool out_step = step >= out0;
             unsigned char *stg = smem + buf * SM::kStage;
             wait_on(&full[buf], (full_phases >> buf) & 1u);
             full_phases ^= 1u << buf;
             const float ds = *reinterpret_cast<const float *>(stg + RC::kGate);
+            if (!xrows) {   // the Y rows read nothing else of the stage
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&free_st[buf]);
+            }
+            wait_on(xy_bar, xy_phase);
+            xy_phase ^= 1;
+            if (*abort_s) break;
+            tc_fence_after();
             if (xrows) {
-                // ---- Delta = U - X -> D (fp16) --------------------------------------
-                wait_on(xy_bar, xy_phase);
-                xy_phase ^= 1;
-                if (*abort_s) break;
-                tc_fence_after();
+                // ---- Delta = U - X -> D (fp16); the previous chunk's P D, issued before
+                //      this [Y; X] by the same thread, has read the old D --------------
 #pragma unroll
                 for (int h16 = 0; h16 < NC; h16 += 16) {
                     float xa[16], xb[16];
@@ -413,8 +406,27 @@ __device__ __forceinline__ void chain_body(
                     mbar_arrive(&free_st[buf]);   // done reading the stage
                     mbar_arrive(d_bar);
                 }
+            } else {
+                // ---- Y -> OY (the output accumulator); this warp read the previous
+                //      chunk's O out of OY at the end of its last step ------------------
+                if (out_step) {
+#pragma unroll
+                    for (int h16 = 0; h16 < NC; h16 += 16) {
+                        float ya[16], yb[16];
+                        tmem_ld16(tmem + lane_base + kColXA + n0 + h16, ya);
+                        tmem_ld16(tmem + lane_base + kColXB + n0 + h16, yb);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) ya[e] += yb[e];
+                        tmem_st16(tmem + lane_base + kColOY + n0 + h16, ya);
+                    }
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(y_bar);
             }
-            // ---- S <- ds S + K~^T D (two token halves) ------------------------------
+            // ---- S <- ds S + K~^T D (token halves in KA and XA) ----------------------
             wait_on(s_bar, s_phase);
             s_phase ^= 1;
             if (*abort_s) break;
@@ -423,7 +435,7 @@ __device__ __forceinline__ void chain_body(
             for (int h16 = 0; h16 < NC; h16 += 16) {
                 float ka[16], kb[16];
                 tmem_ld16(tmem + lane_base + kColKA + n0 + h16, ka);
-                tmem_ld16(tmem + lane_base + kColKB + n0 + h16, kb);
+                tmem_ld16(tmem + lane_base + kColXA + n0 + h16, kb);
                 tmem_wait_ld();
                 uint32_t ss[8];
 #pragma unroll
@@ -437,53 +449,43 @@ __device__ __forceinline__ void chain_body(
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(r_bar);
-            if (xrows) continue;
-            if (step < out0) {
-                // no output during the warm-up: done with the stage
-                if (lane == 0) mbar_arrive(&free_st[buf]);
-                continue;
-            }
-            // ---- output rows: O = Y + P D ------------------------------------------
+            if (xrows || !out_step) continue;
+            // ---- output rows: O = Y + P D out of OY ----------------------------------
             wait_on(pd_bar, pd_phase);
             pd_phase ^= 1;
             if (*abort_s) break;
             tc_fence_after();
             float o[NC];
 #pragma unroll
-            for (int h16 = 0; h16 < NC; h16 += 16) {
-                float ya[16], yb[16];
-                tmem_ld16(tmem + lane_base + kColXA + n0 + h16, ya);
-                tmem_ld16(tmem + lane_base + kColXB + n0 + h16, yb);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) o[h16 + e] = ya[e] + yb[e];
-            }
+            for (int h16 = 0; h16 < NC; h16 += 16) tmem_ld16(tmem + lane_base + kColOY + n0 + h16, o + h16);
+            tmem_wait_ld();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(o_read);
-            // stage the tile for the storer over this stage's [Q~; W] area (the
-            // products are done with it); both directions of a bidirectional scan
-            // add up in fp32
-            unsigned char *ob = stg + RC::kQW;
-            if (sizeof(Tout) == 4 || out.mode == kOutPair) {
+            // stage the tile in the output buffer once the store of the tile before
+            // has read it (o_free completes once per tile; the k-th output tile
+            // waits for the (k-1)-th completion, so it is never two phases behind)
+            {
+                const int k = step - out0;
+                if (k > 0) wait_on(o_free, (uint32_t)((k - 1) & 1));
+                if (*abort_s) break;
+                unsigned char *ob = smem + SM::kO;
+                if (sizeof(Tout) == 4 || out.mode == kOutPair) {
 #pragma unroll
-                for (int q = 0; q < NC / 4; ++q)
-                    *reinterpret_cast<float4 *>(ob + out_stage_off<float>(r, n0 + 4 * q)) =
-                        make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-            } else {
+                    for (int q = 0; q < NC / 4; ++q)
+                        *reinterpret_cast<float4 *>(ob + out_stage_off<float>(r, n0 + 4 * q)) =
+                            make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+                } else {
 #pragma unroll
-                for (int q = 0; q < NC / 8; ++q) {
-                    uint4 w;
-                    w.x = pack_bf16(o[8 * q], o[8 * q + 1]); w.y = pack_bf16(o[8 * q + 2], o[8 * q + 3]);
-                    w.z = pack_bf16(o[8 * q + 4], o[8 * q + 5]); w.w = pack_bf16(o[8 * q + 6], o[8 * q + 7]);
-                    *reinterpret_cast<uint4 *>(ob + out_stage_off<Tout>(r, n0 + 8 * q)) = w;
+                    for (int q = 0; q < NC / 8; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16(o[8 * q], o[8 * q + 1]); w.y = pack_bf16(o[8 * q + 2], o[8 * q + 3]);
+                        w.z = pack_bf16(o[8 * q + 4], o[8 * q + 5]); w.w = pack_bf16(o[8 * q + 6], o[8 * q + 7]);
+                        *reinterpret_cast<uint4 *>(ob + out_stage_off<Tout>(r, n0 + 8 * q)) = w;
+                    }
                 }
+                fence_async_shared();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(o_bar);
             }
-            fence_async_shared();
-            // o_bar completes one phase per tile: not before the storer has seen the last
-            if (step > out0) { wait_on(o_seen, os_phase); os_phase ^= 1; }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(o_bar);
         }
         float *state_out = dir ? states.out[1] : states.out[0];
         if (!*abort_s && state_out && we == nC) {
@@ -503,6 +505,7 @@ __device__ __forceinline__ void chain_body(
         mbar_wait(s_bar, 0, 64);
         mbar_wait(pd_bar, 0, 64);
         mbar_wait(xy_bar, 0, 64);
+        mbar_wait(y_bar, 0, 64);
     }
     tc_fence_before();
     __syncthreads();
@@ -517,8 +520,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_o, const unsigned char *__re
              const ChainStates states, const ChainOut<Tout> out, const ChainSeg seg, int H, int nC,
              unsigned int *__restrict__ err)
 {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    if (smem_u32(smem_raw) & 1023u) {   // no slack was allocated for aligning it here
+        if (threadIdx.x == 0 && err) atomicAdd(err, 1u);
+        return;
+    }
+    unsigned char *smem = smem_raw;
     chain_body<DV, Tout>(&tm_o, recs, states, out, seg, nullptr, H, nC, blockIdx.x, blockIdx.y, blockIdx.z,
                          gridDim.y, smem, err);
 }

@@ -28,10 +28,10 @@ struct FusedPrepSmem {
     static constexpr int kBytes = kCtl + 16;
 };
 
+// (the dynamic shared memory is 1024-aligned, checked at run time)
 template <int DV>
 constexpr int fused_smem_alloc() {
-    return (ChainSmem<DV>::kAlloc > FusedPrepSmem<DV>::kBytes + 1024) ? ChainSmem<DV>::kAlloc
-                                                                       : FusedPrepSmem<DV>::kBytes + 1024;
+    return ChainSmem<DV>::kAlloc > FusedPrepSmem<DV>::kBytes ? ChainSmem<DV>::kAlloc : FusedPrepSmem<DV>::kBytes;
 }
 
 // grid n_chain + n_prep CTAs (cooperative), block kChainThreads.
@@ -46,8 +46,12 @@ fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
              int n_chain, unsigned int *__restrict__ err)
 {
     static_assert(kChainThreads >= 2 * kPrepThreads, "two prep pipelines per CTA");
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    if (smem_u32(smem_raw) & 1023u) {   // no slack was allocated for aligning it here
+        if (threadIdx.x == 0 && err) atomicAdd(err, 1u);
+        return;
+    }
+    unsigned char *smem = smem_raw;
     if ((int)blockIdx.x < n_chain) {
         const int i = blockIdx.x;
         chain_body<DV, Tout>(&tm_o, recs, states, out, seg, ready, H, nC, i % seg.G, (i / seg.G) % nbh,
