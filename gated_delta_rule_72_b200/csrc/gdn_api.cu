@@ -190,10 +190,11 @@ gdn_status dispatch_out(const Args &a, int bidir) {
                              : dispatch_dims<Tin, __nv_bfloat16>(a, bidir);
 }
 
-// The tensor-core path takes bf16 inputs with d_k = 128; everything else runs
-// on the CUDA-core (fp32) path.
+// The tensor-core path takes bf16 inputs (d_k = 64 runs as 128 with zero
+// columns: the key and query tiles are loaded past their width, which reads
+// zeros); fp32 inputs run on the CUDA-core (fp32) path.
 bool use_tc(gdn_dtype dt, int dk, int dv) {
-    return dt == GDN_BF16 && dk == 128 && (dv == 128 || dv == 64);
+    return dt == GDN_BF16 && (dk == 128 || dk == 64) && (dv == 128 || dv == 64);
 }
 
 size_t tc_record_bytes(int dv) {
@@ -427,8 +428,8 @@ bool cooperative_supported() {
 template <int DV, typename Tout>
 gdn_status run_tc(const Args &a, int bidir) {
     CUtensorMap mk, mq, mv;
-    if (!encode_map(&mk, a.k, a.B, a.T, a.H, 128, 64, 128) ||
-        !encode_map(&mq, a.q, a.B, a.T, a.H, 128, 64, 128) ||
+    if (!encode_map(&mk, a.k, a.B, a.T, a.H, a.dk, 64, 128) ||
+        !encode_map(&mq, a.q, a.B, a.T, a.H, a.dk, 64, 128) ||
         !encode_map(&mv, a.v, a.B, a.T, a.H, DV, 64, 128))
         return GDN_ERR_CUDA;
     unsigned int *err = timeout_counter();
@@ -461,6 +462,7 @@ gdn_status run_tc(const Args &a, int bidir) {
     CUtensorMap mo;
     if (!encode_out_map(&mo, target, a, DV, f32_out || bidir)) return GDN_ERR_CUDA;
     gdn::tc2::ChainStates states{};
+    states.dk = a.dk;
     states.in[0] = a.state_in;
     states.out[0] = a.state_out;
     if (bidir) {

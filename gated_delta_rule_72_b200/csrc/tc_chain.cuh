@@ -92,11 +92,15 @@ constexpr int kChainThreads = 20 * 32;
 
 enum OutMode { kOutStore = 0, kOutPair = 1 };
 
-// Initial and final states per direction ([B, H, d_k, d_v] fp32 each; null:
+// Initial and final states per direction ([B, H, dk, d_v] fp32 each; null:
 // zero / not written).  Direction 0 is the causal scan, 1 the reverse one.
+// dk is the caller's key dimension (64 or 128); the chain always runs 128
+// rows, those past dk staying zero (the prep pads keys and queries with zero
+// columns).
 struct ChainStates {
     const float *in[2];
     float *out[2];
+    int dk;
 };
 
 // Output of a chain.  kOutStore: tm_o maps o ([B, T, H, DV], Tout), each
@@ -223,7 +227,8 @@ __device__ __forceinline__ void chain_body(
     float S[NC];
     if (warp < 16) {
         const float *state_in = (w0 == 0) ? (dir ? states.in[1] : states.in[0]) : nullptr;
-        const float *src = state_in ? state_in + ((size_t)bh * kDK + d_row) * DV + n0 : nullptr;
+        const float *src = (state_in && d_row < states.dk) ? state_in + ((size_t)bh * states.dk + d_row) * DV + n0
+                                                           : nullptr;
 #pragma unroll
         for (int n = 0; n < NC; ++n) S[n] = src ? src[n] : 0.f;
 #pragma unroll
@@ -488,8 +493,8 @@ __device__ __forceinline__ void chain_body(
             }
         }
         float *state_out = dir ? states.out[1] : states.out[0];
-        if (!*abort_s && state_out && we == nC) {
-            float *dst = state_out + ((size_t)bh * kDK + d_row) * DV + n0;
+        if (!*abort_s && state_out && we == nC && d_row < states.dk) {
+            float *dst = state_out + ((size_t)bh * states.dk + d_row) * DV + n0;
 #pragma unroll
             for (int n = 0; n < NC; n += 4)
                 *reinterpret_cast<float4 *>(dst + n) = make_float4(S[n], S[n + 1], S[n + 2], S[n + 3]);

@@ -603,7 +603,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             int nC, int nbh, int ndir, PrepOrder po, unsigned int *__restrict__ err)
 {
     using SM = PrepSmem<DV>;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + SM::kCtl);
     if ((threadIdx.x >> 5) == 0) {

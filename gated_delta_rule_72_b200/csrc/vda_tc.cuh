@@ -51,7 +51,7 @@ vda_gram_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 {
     using SM = GramTcSmem<DV>;
     constexpr int NB = 2 * DV;                             // columns of the B part
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::kBar);
     uint64_t *freeb = full + 2;
@@ -245,7 +245,7 @@ vda_readout_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const unsigned c
 {
     using SM = ReadTcSmem<DV>;
     constexpr int NB = 2 * DV;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *loaded = reinterpret_cast<uint64_t *>(smem + SM::kBar);
     uint64_t *done = loaded + 1;

@@ -35,16 +35,35 @@ def test_tiny_workload():
 SHAPES = [(64, 64), (128, 128), (64, 128), (128, 64)]
 
 
+def _kernel_family(names):
+    """'token', 'tc' or 'simt': which path the kernels recorded belong to."""
+    fams = {"token" if n == "token_step" else n.split("_")[0] for n in names}
+    assert len(fams) == 1, names
+    return fams.pop()
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("dk,dv", SHAPES)
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 200])
 def test_causal_shapes(dtype, dk, dv, T):
+    """Causal scans with state in and out; bf16 inputs run on the tensor
+    cores for either key width (d_k = 64 padded to 128 with zero columns),
+    fp32 inputs on the CUDA cores (short calls may take the token path)."""
     B, H = 2, 3
     inp = inputs.generate(B, T, H, dk, dv, dtype, seed=1000 + T + dk + dv)
     s0 = _state(B, H, dk, dv, seed=T)
     d = to_dev(inp)
-    o, s = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"], s0.cuda())
-    torch.cuda.synchronize()
+    gdn.gdn_set_kernel_timing(1)
+    gdn.gdn_read_kernel_timing()
+    try:
+        o, s = gdn.scan_causal(d["q"], d["k"], d["v"], d["alpha"], d["beta"], s0.cuda())
+        torch.cuda.synchronize()
+        fam = _kernel_family(gdn.gdn_read_kernel_timing())
+    finally:
+        gdn.gdn_set_kernel_timing(0)
+    assert fam in ("token", "tc" if dtype == "bf16" else "simt"), fam
+    if T > 64:
+        assert fam == ("tc" if dtype == "bf16" else "simt"), fam
     o_ref, s_ref = oracle_heads(inp, state_in=s0)
     tol = TOL[DT[dtype]]
     assert rel_err(o, o_ref) <= tol
@@ -103,14 +122,23 @@ def test_short_call_threshold_switches_path():
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (128, 64)])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (128, 64), (64, 128)])
 @pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 130, 257])
 def test_bidir_shapes(dtype, dk, dv, T):
+    """Bidirectional scans: bf16 inputs on the tensor cores for both key
+    widths, fp32 inputs on the CUDA cores."""
     B, H = 1, 3
     inp = inputs.generate(B, T, H, dk, dv, dtype, seed=2000 + T + dk)
     d = to_dev(inp)
-    o = gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
-    torch.cuda.synchronize()
+    gdn.gdn_set_kernel_timing(1)
+    gdn.gdn_read_kernel_timing()
+    try:
+        o = gdn.scan_bidir(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+        torch.cuda.synchronize()
+        fam = _kernel_family(gdn.gdn_read_kernel_timing())
+    finally:
+        gdn.gdn_set_kernel_timing(0)
+    assert fam == ("tc" if dtype == "bf16" else "simt"), fam
     o_ref, _ = oracle_heads(inp, mode="bidir")
     assert rel_err(o, o_ref) <= TOL[DT[dtype]]
 

@@ -29,7 +29,7 @@ def _state(B, H, dk, dv, seed):
 
 @pytest.mark.parametrize("bidir", [False, True])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64)])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64), (64, 128)])
 @pytest.mark.parametrize("F,U", [(3, 40), (2, 130), (5, 1)])
 def test_vda_parity(bidir, dtype, dk, dv, F, U):
     B, H = 2, 3
@@ -80,3 +80,23 @@ def test_vda_frames_equal_token_scan_for_one_token_frames():
     torch.cuda.synchronize()
     assert rel_err(o1, o2.double().cpu().numpy()) <= 1e-4
     assert rel_err(s1, s2.double().cpu().numpy()) <= 1e-4
+
+
+def test_vda480_full_frame_length():
+    """The benchmarked frame-wise workload as timed (B=1, H=12, 21 frames of
+    1,560 tokens, d = 128, bf16, bidirectional): two sampled heads against the
+    oracle, every output of those heads."""
+    w = inputs.WORKLOADS["vda480"]
+    inp = inputs.workload_inputs(w)
+    af = inputs.frame_alpha(inp["alpha"], w.frame)
+    d = to_dev(inp)
+    o = gdn.vda_scan(d["q"], d["k"], d["v"], af.cuda(), d["beta"], w.frame, bidir=True)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o).all()
+    heads = [2, 9]
+    sel = lambda t: t[:, :, heads].contiguous()
+    o_ref, _, _ = oracle.vda_scan(sel(inp["q"]), sel(inp["k"]), sel(inp["v"]), sel(af), sel(inp["beta"]), w.frame,
+                                  mode="bidir")
+    err = rel_err(o.cpu()[:, :, heads], o_ref)
+    print("vda480 parity max|o - o_oracle| / rms(o_oracle) = %.3e" % err)
+    assert err <= TOL[torch.bfloat16]
