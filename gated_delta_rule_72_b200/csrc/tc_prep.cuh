@@ -311,15 +311,24 @@ __device__ __forceinline__ void prep_pipeline(
             if (ln < 64) {
                 const float br = beta_s[r], gr = g_s[r];
                 const float eA = br * Xsm[64 + r * 4 + kA], eB = br * Xsm[64 + r * 4 + kB];
-                float kk = 0.f;                          // |k_r|^2 (diagonal of the Gram)
+                // (the decay test is task-uniform: one loop or the other runs)
+                if (fast) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int s = rev ? 63 - (f0 + e) : f0 + e;
-                    const float w = fast ? (e < 16 ? eA : eB) * facs[s] : br * __expf(gr - g_s[s]);
-                    Lsm[r * 65 + s] = s < r ? w * G[e] : 0.f;
-                    if (f0 + e == fl) kk = G[e];
+                    for (int e = 0; e < 32; ++e) {
+                        const int s = rev ? 63 - (f0 + e) : f0 + e;
+                        Lsm[r * 65 + s] = s < r ? (e < 16 ? eA : eB) * facs[s] * G[e] : 0.f;
+                    }
+                } else {
+#pragma unroll 4
+                    for (int e = 0; e < 32; ++e) {
+                        const int s = rev ? 63 - (f0 + e) : f0 + e;
+                        Lsm[r * 65 + s] = s < r ? br * __expf(gr - g_s[s]) * G[e] : 0.f;
+                    }
                 }
                 if (half == (fl >> 5)) {   // warps 0 and 5 hold the diagonal of rows 0-31 / 32-63
+                    float kk = 0.f;        // |k_r|^2: the Gram's diagonal, column fl - f0 = lane
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) kk = e == lane ? G[e] : kk;
                     float term = __logf(fmaxf(1.f, fabsf(1.f - br * kk)));
 #pragma unroll
                     for (int d = 16; d > 0; d >>= 1) term += __shfl_xor_sync(0xffffffffu, term, d);
@@ -331,13 +340,22 @@ __device__ __forceinline__ void prep_pipeline(
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     float v[8];
+                    if (fast) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int f = f0 + cc * 8 + e;
-                        const int s = rev ? 63 - f : f;
-                        const bool keep = rev ? (s < r) : (s <= r);
-                        const float w = fast ? (cc < 2 ? eA : eB) * facs[s] : __expf(gq - g_s[s]);
-                        v[e] = keep ? w * G[cc * 8 + e] : 0.f;
+                        for (int e = 0; e < 8; ++e) {
+                            const int f = f0 + cc * 8 + e;
+                            const int s = rev ? 63 - f : f;
+                            const bool keep = rev ? (s < r) : (s <= r);
+                            v[e] = keep ? (cc < 2 ? eA : eB) * facs[s] * G[cc * 8 + e] : 0.f;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int f = f0 + cc * 8 + e;
+                            const int s = rev ? 63 - f : f;
+                            const bool keep = rev ? (s < r) : (s <= r);
+                            v[e] = keep ? __expf(gq - g_s[s]) * G[cc * 8 + e] : 0.f;
+                        }
                     }
                     uint4 p;
                     p.x = pack_f16(v[0], v[1]); p.y = pack_f16(v[2], v[3]);
