@@ -17,18 +17,18 @@
 // 130 cycles whatever N is up to 256, so the halves run side by side.
 //
 // TMEM (4 x DV columns): XA, XB hold the two K halves of [Y; X]; KA and then
-// XA (once read) the two token halves of K~^T D; OY holds O: the Y rows copy
-// Y there (tcgen05.st) while the X rows form D, and P D accumulates onto it.
-// So the next chunk's [Q~; W] S waits only for the state, never for the
-// output, and P D stays off the chain's critical path.
+// XA (once its X rows are read) the two token halves of K~^T D; OY holds O: a
+// second [Q~; W] S product (one stream, issued while the X rows form D) puts
+// Y there and P D accumulates onto it.  So the next chunk's [Q~; W] S waits
+// only for the state, and the output stays off the chain's critical path.
 //
 // Roles (20 warps).  The 16 epilogue warps cover the 128 TMEM lanes four
 // times (warp w reads lane quarter w % 4, columns DV/4 * (w / 4) .. +DV/4-1):
 //   quarters 2, 3 (X rows)  Delta = U - X -> D             (critical path)
-//   quarters 0, 1 (Y rows)  Y -> OY, then O = OY -> staged output tile
+//   quarters 0, 1 (Y rows)  O = OY -> staged output tile
 //   all                     S <- ds S + K~^T D, thread = one row of S
 // Warps 16 and 17 issue the two halves of the chain's products (16 also
-// P D) and warp 18 loads the records (one bulk copy per chunk,
+// the output's Y and P D) and warp 18 loads the records (one bulk copy per chunk,
 // double-buffered).  A stage is free again once both issuers' products are
 // done and every epilogue warp has read it.  The Y rows write the output
 // straight to global memory from registers.  Roles meet on mbarriers; every
@@ -36,7 +36,8 @@
 // kernel wind down.  A
 // tcgen05.commit covers every earlier MMA of its issuing thread, so the
 // [Y; X] product of a chunk completing also means that thread's P D of the
-// chunk before has completed (and no longer reads D).
+// chunk before has completed (and no longer reads D), and K~^T D completing
+// means the output's Y product has read S.
 //
 // Sequence parallelism.  A chain of n chunks is cut into G segments of L
 // chunks of the walk; segment g emits the outputs of walk steps
@@ -152,7 +153,7 @@ __device__ __forceinline__ void chain_body(
     uint64_t *s_bar = bars + 6;        // K~^T D complete, 2 commits               (-> epilogue)
     uint64_t *r_bar = bars + 7;        // S rewritten, 16 warps                    (-> A, B)
     uint64_t *pd_bar = bars + 8;       // Y + P D complete in OY, 1 commit          (-> Y warps)
-    uint64_t *y_bar = bars + 9;        // Y moved to OY (Y lanes of XA, XB free), 8 Y warps (-> A, B)
+    uint64_t *y_bar = bars + 9;        // O read out of OY, 8 Y warps               (-> A)
     uint64_t *o_bar = bars + 10;       // output tile staged, 8 Y warps            (-> storer)
     uint64_t *o_free = bars + 11;      // output buffer read by its store          (storer -> Y warps)
     uint32_t *tmem_base_s = reinterpret_cast<uint32_t *>(smem + SM::kCtl);
@@ -285,7 +286,7 @@ __device__ __forceinline__ void chain_body(
         __syncwarp();
     } else if (warp == 16 || warp == 17) {
         // ===== issuers A (warp 16) and B (warp 17): one half of each chain product;
-        // A also P D onto OY
+        // A also the output's [Q~; W] S into OY and P D onto it
         if (lane == 0) {
             const int part = warp - 16;
             const uint32_t colX = part ? kColXB : kColXA;
@@ -307,11 +308,21 @@ __device__ __forceinline__ void chain_body(
                     mma_bf16(tmem + colX, a, adv(dS, (part * 4 + k) * 2048), idXY, k > 0);
                 }
                 mma_commit(xy_bar);
-                // D written (X rows read) and Y moved to OY (Y rows read)
+                if (part == 0 && step >= out0) {
+                    // the output's Y = [Q~; W] S into OY (rows 64-127 unused), once the
+                    // previous chunk's O has been read out of OY
+                    if (step > out0) { wait_on(y_bar, y_phase); y_phase ^= 1; }
+                    if (*abort_s) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint64_t a = sdesc_sw128(st + RC::kQW + (k >> 2) * 16384 + (k & 3) * 32);
+                        mma_bf16(tmem + kColOY, a, adv(dS, k * 2048), idXY, k > 0);
+                    }
+                }
+                // D written (X rows of XA, XB read)
                 wait_on(d_bar, d_phase);
                 d_phase ^= 1;
-                wait_on(y_bar, y_phase);
-                y_phase ^= 1;
                 if (*abort_s) break;
                 tc_fence_after();
                 // K~^T D half: tokens 32*part .. +31
@@ -379,11 +390,11 @@ __device__ __forceinline__ void chain_body(
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&free_st[buf]);
             }
-            wait_on(xy_bar, xy_phase);
-            xy_phase ^= 1;
-            if (*abort_s) break;
-            tc_fence_after();
             if (xrows) {
+                wait_on(xy_bar, xy_phase);
+                xy_phase ^= 1;
+                if (*abort_s) break;
+                tc_fence_after();
                 // ---- Delta = U - X -> D (fp16); the previous chunk's P D, issued before
                 //      this [Y; X] by the same thread, has read the old D --------------
 #pragma unroll
@@ -411,25 +422,6 @@ __device__ __forceinline__ void chain_body(
                     mbar_arrive(&free_st[buf]);   // done reading the stage
                     mbar_arrive(d_bar);
                 }
-            } else {
-                // ---- Y -> OY (the output accumulator); this warp read the previous
-                //      chunk's O out of OY at the end of its last step ------------------
-                if (out_step) {
-#pragma unroll
-                    for (int h16 = 0; h16 < NC; h16 += 16) {
-                        float ya[16], yb[16];
-                        tmem_ld16(tmem + lane_base + kColXA + n0 + h16, ya);
-                        tmem_ld16(tmem + lane_base + kColXB + n0 + h16, yb);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) ya[e] += yb[e];
-                        tmem_st16(tmem + lane_base + kColOY + n0 + h16, ya);
-                    }
-                    tmem_wait_st();
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(y_bar);
             }
             // ---- S <- ds S + K~^T D (token halves in KA and XA) ----------------------
             wait_on(s_bar, s_phase);
@@ -465,6 +457,8 @@ __device__ __forceinline__ void chain_body(
             for (int h16 = 0; h16 < NC; h16 += 16) tmem_ld16(tmem + lane_base + kColOY + n0 + h16, o + h16);
             tmem_wait_ld();
             tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(y_bar);   // OY may take the next chunk's Y
             // stage the tile in the output buffer once the store of the tile before
             // has read it (o_free completes once per tile; the k-th output tile
             // waits for the (k-1)-th completion, so it is never two phases behind)
