@@ -83,7 +83,8 @@ __device__ __forceinline__ bool prep_task(const PrepOrder &po, int t, int nbh, i
 
 // One prep pipeline: 256 threads (ptid 0..255) with their own 1024-aligned
 // shared-memory area `smem` (PrepSmem<DV>), 256 TMEM columns from `tmem` and
-// named barrier `bar_id`; it walks tasks first_task, first_task + stride, ...
+// named barriers `bar_id` (all 256 threads), `aux_id` (warps 0-1) and
+// `aux_id + 1` (warps 0-3); it walks tasks first_task, first_task + stride, ...
 // (po order).  With `ready` non-null, each record's flag is set (release) once
 // its stores have landed, for a chain kernel that runs alongside.
 template <int DV>
@@ -91,7 +92,7 @@ __device__ __forceinline__ void prep_pipeline(
     const CUtensorMap *tm_k, const CUtensorMap *tm_q, const CUtensorMap *tm_v,
     const float *__restrict__ alpha, const float *__restrict__ beta, unsigned char *__restrict__ recs,
     float *__restrict__ lb, unsigned int *__restrict__ ready, int T, int H, int nC, int nbh, int ndir,
-    PrepOrder po, int first_task, int task_stride, unsigned char *smem, uint32_t tmem, int ptid, int bar_id,
+    PrepOrder po, int first_task, int task_stride, unsigned char *smem, uint32_t tmem, int ptid, int bar_id, int aux_id,
     unsigned int *__restrict__ err)
 {
     using SM = PrepSmem<DV>;
@@ -119,6 +120,8 @@ __device__ __forceinline__ void prep_pipeline(
     const uint32_t sbase = smem_u32(smem);
     const int ntasks = po.L * po.G * ndir * nbh;
     auto psync = [&]() { asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory"); };
+    auto sync64 = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(aux_id) : "memory"); };     // warps 0-1
+    auto sync128 = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(aux_id + 1) : "memory"); };  // warps 0-3
 
     if (tid == 0) {
         mbar_init(tma_bar, 1);
@@ -242,8 +245,8 @@ __device__ __forceinline__ void prep_pipeline(
             g_s[2 * lane] = ex + a0;
             g_s[2 * lane + 1] = ex + a0 + a1;
         }
-        psync();
-        if (tid < 64) {
+        if (tid < 64) {   // only warps 0 and 1 use the prefix sums before the next barrier
+            sync64();
             const float gr = g_s[tid], gl = g_s[63];
             dq_s[tid] = rev ? (tid > 0 ? __expf(g_s[tid - 1]) : 1.f) : __expf(gr);
             dkk_s[tid] = __expf(gl - gr);
@@ -428,8 +431,8 @@ __device__ __forceinline__ void prep_pipeline(
             }
             float *xb = Xsm + b2 * 256 + (2 * ti) * 16 + 2 * tj;
             xb[0] = x00; xb[1] = x01; xb[16] = x10; xb[17] = x11;
+            sync128();      // level 2 is warps 0-3 alone
         }
-        psync();
         if (tid < 128) {   // level 2, T_10 = -T_11 X
             const int b2 = tid >> 6, ti = (tid >> 3) & 7, tj = tid & 7, base = 32 * b2;
             const int a = base + 16 + 2 * ti, bc = base + 2 * tj;
@@ -494,7 +497,6 @@ __device__ __forceinline__ void prep_pipeline(
             Tsm[a * 65 + bc] = -y00; Tsm[a * 65 + bc + 1] = -y01;
             Tsm[(a + 1) * 65 + bc] = -y10; Tsm[(a + 1) * 65 + bc + 1] = -y11;
         }
-        psync();
         // the P store has read its staging area (the T images go there next)
         if (tid == 0) bulk_wait_read_all();
         psync();
@@ -633,7 +635,7 @@ prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     tc_fence_after();
     const uint32_t tmem = *tmem_base_s;
     prep_pipeline<DV>(&tm_k, &tm_q, &tm_v, alpha, beta, recs, lb, nullptr, T, H, nC, nbh, ndir, po, blockIdx.x,
-                      gridDim.x, smem, tmem, threadIdx.x, 0, err);
+                      gridDim.x, smem, tmem, threadIdx.x, 0, 1, err);
     __syncthreads();
     if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, kPrepTmemCols);
 }

@@ -46,6 +46,18 @@
  *           Rounding to bf16 alone moves max|o|/rms(o) by up to 2^-8 times
  *           max|o|/rms(o), which on long sequences is several 1e-2, so the
  *           fp32 output is the one that carries the accuracy of the scan.
+ *  Paths    fp32 inputs run on the CUDA cores in fp32 (max|o - exact| /
+ *           rms(o) near 1e-6).  bf16 inputs (dk = 64 or 128; 64 runs as 128
+ *           with zero columns) run on the tensor cores: the chunk algebra's
+ *           products take fp16 operands (each computed operand rounded once;
+ *           T diag(beta) as a bf16 hi/lo pair) with fp32 accumulation, about
+ *           3e-3 .. 8e-3 of rms(o) on sequences of 16k to 262k tokens.  fp16
+ *           holds magnitudes up to 65504: the state and the values must stay
+ *           below that (they do for unit-norm keys and values of moderate
+ *           size; the scan is linear in v and the state, so larger inputs can
+ *           be scaled down and the output scaled back).  Long chunk walks are
+ *           cut into segments that run in parallel (gdn_set_chain_segments),
+ *           which drops contributions below 2^-30 of the state.
  */
 #ifndef GDN_H
 #define GDN_H
@@ -157,7 +169,8 @@ GDN_API gdn_status gdn_step(const void *q, const void *k, const void *v,
  *   - Arguments whose gdn_workspace_size(..., bidir = 0) exceeds
  *     GDN_NOALLOC_SCRATCH_BYTES are rejected with GDN_ERR_WORKSPACE before
  *     any launch (for d_k = d_v = 128 and bf16 inputs, whose workspace is
- *     one 66,560-byte record per chunk-head, that is B*H*ceil(T/64) > 1,008).
+ *     one 73,856-byte record, a flag and a bound per chunk-head, that is
+ *     B*H*ceil(T/64) > 908).
  *   - All calls share the one array and it keeps the last call's contents;
  *     nothing in it needs to start at zero (every scratch byte a call reads
  *     was written earlier by the same call, in stream order).  Calls that
@@ -199,9 +212,10 @@ GDN_API int gdn_set_short_call_tokens(int max_t);
 
 /*
  * gdn_set_chain_segments -- how many segments the tensor-core path cuts each
- * (b, h, direction) chunk walk into (sequence parallelism; bf16 inputs with
- * d_k = 128).  g < 1: automatic (the default): enough segments to occupy the
- * SMs, at least 16 chunks each; g >= 1: g segments (at most one per chunk).
+ * (b, h, direction) chunk walk into (sequence parallelism; bf16 inputs).
+ * g < 1: automatic (the default): enough segments to occupy the SMs with one
+ * wave of chain CTAs, at least 6 chunks each; g >= 1: g segments (at most one
+ * per chunk).
  * A segment other than the first starts from a zero state some chunks before
  * its first output, at the first chunk boundary where the 2-norm bound of the
  * skipped state maps, the product over the skipped tokens of
@@ -235,8 +249,13 @@ GDN_API int gdn_set_chain_segments(int g);
  *   state_out_bwd the reverse R_{F+1} / R_1 (used only when bidir; NULL: zero /
  *   not written), with the overlap rules of gdn_scan_bidir_states.
  *   Workspace: gdn_vda_workspace_size bytes, 256-byte aligned.  F = 0 passes
- *   the states through.  All arithmetic in fp32 (CUDA cores): a Cholesky
- *   factorisation of I + A_f per frame and head.
+ *   the states through.  Two paths: fp32 inputs (or dk = 64) run every step in
+ *   fp32 on the CUDA cores; bf16 inputs with dk = 128 take the frame Gram
+ *   [A_f | B_f] and the readout on the tensor cores (bf16 keys and queries
+ *   exact, the beta-scaled keys and values and the states as bf16 hi/lo
+ *   pairs, fp32 accumulation).  Either way (I + A_f)^{-1} comes from an fp32
+ *   Cholesky factorisation per frame and head, and the state recurrence is
+ *   fp32 on the CUDA cores.
  */
 GDN_API gdn_status gdn_vda_scan(const void *q, const void *k, const void *v, const float *alpha_frame,
                                 const float *beta, const float *state_in, const float *state_in_bwd,
