@@ -20,8 +20,8 @@ runs the same workload as an independent problem (weak scaling, no data-path
 collective) and the max over ranks is used.
 
 Extra keys: `roofline` (the dominant kernel's algorithmic bytes or FLOPs per
-launch over its mean CUDA-event duration in the same timed region, against
-the measured peak), `cpu_baseline` (the FP64 oracle on a bounded sample, on
+launch over its mean CUDA-event duration, from a second pass of the same
+steps with an event pair around every launch, against the measured peak), `cpu_baseline` (the FP64 oracle on a bounded sample, on
 the host cores; rank 0 at N = 1), `e2e` (the same metric through the Python
 API with the inputs copied from pinned host memory and the output and state
 read back inside the timed region), `clocks` (nvidia-smi samples taken during
@@ -459,15 +459,19 @@ def measure(torch, gdn, w, device, args, dist, rank, clocks=True):
         while time.time() < t_end:
             step.run()
             torch.cuda.synchronize()
-    gdn.gdn_read_kernel_timing()                  # drop anything recorded so far
     n0 = gdn.gdn_launch_count()
-    gdn.gdn_set_kernel_timing(1)
     ms = timed(torch, step.run, step.between, args.steps, dist)
-    gdn.gdn_set_kernel_timing(0)
     launches = gdn.gdn_launch_count() - n0
     clk = sampler.stop() if sampler else None
-    ktimes = gdn.gdn_read_kernel_timing()
     ms = max_over_ranks(torch, dist, ms, device)
+    # the per-kernel breakdown comes from a second pass of the same steps with
+    # an event pair around every launch (kept out of the timed pass above:
+    # the events add host work per launch)
+    gdn.gdn_read_kernel_timing()                  # drop anything recorded so far
+    gdn.gdn_set_kernel_timing(1)
+    timed(torch, step.run, step.between, args.steps, dist)
+    gdn.gdn_set_kernel_timing(0)
+    ktimes = gdn.gdn_read_kernel_timing()
     units = w.token_heads                          # per GPU per step
     peaks, peak_src = load_peaks()
     return {"step": step, "ms": ms, "value": whole_job_value(args.gpus, units, ms),
