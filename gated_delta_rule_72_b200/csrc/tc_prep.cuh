@@ -322,7 +322,7 @@ __device__ __forceinline__ void prep_pipeline(
                         Lsm[r * 65 + s] = s < r ? (e < 16 ? eA : eB) * facs[s] * G[e] : 0.f;
                     }
                 } else {
-#pragma unroll 4
+#pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int s = rev ? 63 - (f0 + e) : f0 + e;
                         Lsm[r * 65 + s] = s < r ? br * __expf(gr - g_s[s]) * G[e] : 0.f;
@@ -410,7 +410,6 @@ __device__ __forceinline__ void prep_pipeline(
                 unsigned char *dst = rec + (is_k ? RC::kK + (blk & 1) * 8192 : RC::kQW + (blk & 1) * 16384) + within;
                 *reinterpret_cast<uint4 *>(dst) = make_uint4(o16[0], o16[1], o16[2], o16[3]);
             }
-            __threadfence();   // the record's Q~ and K~ are published with its flag
         }
         psync();
         // off-diagonal blocks by recursive doubling (processing order):
@@ -583,6 +582,13 @@ __device__ __forceinline__ void prep_pipeline(
                 }
             }
             fence_async_shared();
+            // With a chain alongside, the record's Q~ and K~ (plain stores of the
+            // conversion threads) must be visible before its flag is set, at the
+            // next task.  The fence sits here, long after those stores: right
+            // after them it held up each thread's next shared-memory access until
+            // they had drained (about 1.5 K cycles per task).  A standalone prep
+            // needs no fence: the chain kernel starts after it.
+            if (ready) __threadfence();
         }
         tc_fence_before();
         psync();
