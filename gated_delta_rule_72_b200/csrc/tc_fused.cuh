@@ -75,7 +75,7 @@ fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         const int npipes = 2 * ((int)gridDim.x - n_chain);
         prep_pipeline<DV>(&tm_k, &tm_q, &tm_v, alpha, beta, recs, lb, ready, T, H, nC, nbh, ndir, po,
                           2 * ((int)blockIdx.x - n_chain) + pipe, npipes, smem + pipe * FS::kArea,
-                          tmem + pipe * kPrepTmemCols, threadIdx.x & (kPrepThreads - 1), 1 + pipe, 3 + 2 * pipe,
+                          tmem + pipe * kPrepTmemCols, threadIdx.x & (kPrepThreads - 1), 1 + pipe, 3 + pipe,
                           err);
     }
     __syncthreads();

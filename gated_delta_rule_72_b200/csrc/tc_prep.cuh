@@ -28,6 +28,19 @@
 namespace gdn {
 namespace tc2 {
 
+// Gate vectors of one task (fp32, processing order), computed one task ahead.
+struct PrepGate {
+    static constexpr int kG = 0;       // g_r, prefix sums of log alpha
+    static constexpr int kBeta = 64;   // beta_r
+    static constexpr int kDq = 128;    // e^{g_r} (reverse: e^{g_{r-1}}), the query scale
+    static constexpr int kDkk = 192;   // e^{g_63 - g_r}, the key scale of the state update
+    static constexpr int kBg = 256;    // beta_r e^{g_r}
+    static constexpr int kFacs = 320;  // e^{g_16k - g_r}, k = r / 16 (mask decay factors)
+    static constexpr int kFast = 384;  // (int) 1 if every 16-token block decays by less than 80
+    static constexpr int kDs = 385;    // e^{g_63}
+    static constexpr int kFloats = 392;
+};
+
 template <int DV>
 struct PrepSmem {
     static constexpr int kKQ = 32768;                 // [K|Q] x 2 column blocks, 128B swizzle
@@ -35,12 +48,12 @@ struct PrepSmem {
     static constexpr int kStage = kKQ + kVb;          // one stage, 1024-aligned
     static constexpr int kL = kStage;                 // [64][65] fp32
     static constexpr int kT = kL + 64 * 65 * 4;       // [64][65] fp32
-    static constexpr int kX = kT + 64 * 65 * 4;       // 3 x [16][16] fp32
-    static constexpr int kT1 = (kX + 3 * 256 * 4 + 1023) / 1024 * 1024;   // bf16 K-major 64 x 64
+    static constexpr int kX = kT + 64 * 65 * 4;       // 2 x [16][16] fp32 (level-2 scratch)
+    static constexpr int kT1 = (kX + 2 * 256 * 4 + 1023) / 1024 * 1024;   // bf16 K-major 64 x 64
     static constexpr int kT2h = kT1 + 8192;           // T diag(beta), bf16 hi
     static constexpr int kT2l = kT2h + 8192;          // and lo
-    static constexpr int kGate = kT2l + 8192;         // g, beta, dq, dkk, beta e^g
-    static constexpr int kMisc = kGate + 5 * 256;     // key-norm partials [2], record gate [4], task [2][4]
+    static constexpr int kGate = kT2l + 8192;         // two gate buffers (PrepGate), by task parity
+    static constexpr int kMisc = kGate + 2 * 4 * PrepGate::kFloats;   // key-norm partials [2], record gate [4], task [2][4]
     static constexpr int kBar = kMisc + 64;           // tma, mma, gram
     static constexpr int kCtl = kBar + 32;            // tmem base, abort, ds
     static constexpr int kBytes = kCtl + 16;
@@ -83,8 +96,8 @@ __device__ __forceinline__ bool prep_task(const PrepOrder &po, int t, int nbh, i
 
 // One prep pipeline: 256 threads (ptid 0..255) with their own 1024-aligned
 // shared-memory area `smem` (PrepSmem<DV>), 256 TMEM columns from `tmem` and
-// named barriers `bar_id` (all 256 threads), `aux_id` (warps 0-1) and
-// `aux_id + 1` (warps 0-3); it walks tasks first_task, first_task + stride, ...
+// named barriers `bar_id` (all 256 threads) and `aux_id` (warps 0-3); it
+// walks tasks first_task, first_task + stride, ...
 // (po order).  With `ready` non-null, each record's flag is set (release) once
 // its stores have landed, for a chain kernel that runs alongside.
 template <int DV>
@@ -100,18 +113,13 @@ __device__ __forceinline__ void prep_pipeline(
     float *Lsm = reinterpret_cast<float *>(smem + SM::kL);
     float *Tsm = reinterpret_cast<float *>(smem + SM::kT);
     float *Xsm = reinterpret_cast<float *>(smem + SM::kX);
-    float *g_s = reinterpret_cast<float *>(smem + SM::kGate);
-    float *beta_s = g_s + 64;
-    float *dq_s = g_s + 128;
-    float *dkk_s = g_s + 192;
-    float *bg_s = g_s + 256;
+    float *gate_s = reinterpret_cast<float *>(smem + SM::kGate);   // [2][PrepGate::kFloats]
     float *kf_s = reinterpret_cast<float *>(smem + SM::kMisc);        // [2] key-norm terms
     float *rgate_s = reinterpret_cast<float *>(smem + SM::kMisc + 16); // [4] record gate (ds)
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + SM::kBar);
     uint64_t *mma_bar = tma_bar + 1;
     uint64_t *g_bar = tma_bar + 2;     // the two K halves of the Gram product
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + SM::kCtl + 4);
-    float *ds_s = reinterpret_cast<float *>(smem + SM::kCtl + 8);
 
     const int tid = ptid, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;                  // TMEM lane quarter of this warp
@@ -120,8 +128,7 @@ __device__ __forceinline__ void prep_pipeline(
     const uint32_t sbase = smem_u32(smem);
     const int ntasks = po.L * po.G * ndir * nbh;
     auto psync = [&]() { asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory"); };
-    auto sync64 = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(aux_id) : "memory"); };     // warps 0-1
-    auto sync128 = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(aux_id + 1) : "memory"); };  // warps 0-3
+    auto sync128 = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(aux_id) : "memory"); };  // warps 0-3
 
     if (tid == 0) {
         mbar_init(tma_bar, 1);
@@ -171,15 +178,57 @@ __device__ __forceinline__ void prep_pipeline(
             if (err) atomicAdd(err, 1u);
         }
     };
-    // gates of a task, processing order: thread r < 64 loads row r (raw alpha:
-    // the logarithm is taken when the value is used, so the load's latency is
-    // not waited for here)
-    auto load_gates = [&](int dir, int c, int bh, float &al, float &bt) {
+    // Gates of a task, by warp 4, one task ahead: lane l loads rows 2l and 2l+1
+    // (processing order; raw values, so that the loads' latency is not waited
+    // for here) ...
+    auto load_gates = [&](int dir, int c, int bh, float2 &al, float2 &bt) {
         const int b = bh / H, h = bh % H;
-        const int tok = token_of_row(c, tid, dir);
-        const size_t off = ((size_t)b * T + tok) * H + h;
-        al = tok < T ? alpha[off] : 1.f;
-        bt = tok < T ? beta[off] : 0.f;
+        const int t0 = token_of_row(c, 2 * lane, dir), t1 = token_of_row(c, 2 * lane + 1, dir);
+        const size_t o0 = ((size_t)b * T + t0) * H + h, o1 = ((size_t)b * T + t1) * H + h;
+        al.x = t0 < T ? alpha[o0] : 1.f;
+        bt.x = t0 < T ? beta[o0] : 0.f;
+        al.y = t1 < T ? alpha[o1] : 1.f;
+        bt.y = t1 < T ? beta[o1] : 0.f;
+    };
+    // ... and fills the task's gate buffer (PrepGate) from them.
+    auto make_gates = [&](float *gb, float2 al, float2 bt, bool rv) {
+        const float a0 = __logf(al.x), a1 = __logf(al.y);
+        float s = a0 + a1;   // inclusive prefix sum over the lanes of the row-pair sums
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, s, d);
+            if (lane >= d) s += y;
+        }
+        const float ex = s - (a0 + a1);
+        const float g0 = ex + a0, g1 = ex + a0 + a1;                    // rows 2l, 2l+1
+        const float gl = __shfl_sync(0xffffffffu, g1, 31);              // g_63
+        const float gm = __shfl_up_sync(0xffffffffu, g1, 1);            // g_{2l-1}
+        const float gb16 = __shfl_sync(0xffffffffu, g0, lane & ~7);     // g_16k of this row pair's block
+        const int r0 = 2 * lane;
+        gb[PrepGate::kG + r0] = g0;
+        gb[PrepGate::kG + r0 + 1] = g1;
+        gb[PrepGate::kBeta + r0] = bt.x;
+        gb[PrepGate::kBeta + r0 + 1] = bt.y;
+        gb[PrepGate::kDq + r0] = rv ? (lane > 0 ? __expf(gm) : 1.f) : __expf(g0);
+        gb[PrepGate::kDq + r0 + 1] = rv ? __expf(g0) : __expf(g1);
+        gb[PrepGate::kDkk + r0] = __expf(gl - g0);
+        gb[PrepGate::kDkk + r0 + 1] = __expf(gl - g1);
+        gb[PrepGate::kBg + r0] = bt.x * __expf(g0);
+        gb[PrepGate::kBg + r0 + 1] = bt.y * __expf(g1);
+        // Decay factors of the masks without an exponential per entry: for s in
+        // the 16-token block k, e^{g_r - g_s} = e^{g_r - g_16k} e^{g_16k - g_s}.
+        // On the entries the masks keep (16k <= s <= r) the first factor is at
+        // most 1 and the second at most e^(decay over 16 tokens), so both are
+        // finite whenever that decay stays below 80 (else: one exponential per
+        // entry).
+        gb[PrepGate::kFacs + r0] = __expf(gb16 - g0);
+        gb[PrepGate::kFacs + r0 + 1] = __expf(gb16 - g1);
+        const bool ok = (lane & 7) != 7 || gb16 - g1 < 80.f;            // g_16k - g_16k+15
+        const bool fast = __all_sync(0xffffffffu, ok);
+        if (lane == 0) {
+            reinterpret_cast<int *>(gb)[PrepGate::kFast] = fast ? 1 : 0;
+            gb[PrepGate::kDs] = __expf(gl);
+        }
     };
 
     int t = 0;   // thread 0: index of the current task
@@ -194,9 +243,12 @@ __device__ __forceinline__ void prep_pipeline(
         const int i = e >> 6, jj = e & 63;
         if ((jj >> 4) > (i >> 4)) Tsm[i * 65 + jj] = 0.f;
     }
-    psync();
-    float al_n = 1.f, bt_n = 0.f;
-    if (tid < 64 && desc[0]) load_gates(desc[1], desc[2], desc[3], al_n, bt_n);
+    psync();   // (desc[0] is set)
+    float2 al_n = make_float2(1.f, 1.f), bt_n = make_float2(0.f, 0.f);   // warp 4: the next task's raw gates
+    if (warp == 4 && desc[0]) {
+        load_gates(desc[1], desc[2], desc[3], al_n, bt_n);
+        make_gates(gate_s, al_n, bt_n, desc[1] != 0);
+    }
     uint32_t tma_phase = 0, mma_phase = 0, g_phase = 0;
     unsigned int *pending_flag = nullptr;   // thread 0: ready flag of the last record stored
     const uint32_t st_addr = sbase;
@@ -214,13 +266,14 @@ __device__ __forceinline__ void prep_pipeline(
             put_desc(nxt, tn);
         }
 
-        if (tid < 64) { g_s[tid] = __logf(al_n); beta_s[tid] = bt_n; }
+        const float *gb = gate_s + slot * PrepGate::kFloats;   // this task's gates (made one task ahead)
+        const float *g_s = gb + PrepGate::kG, *beta_s = gb + PrepGate::kBeta, *dq_s = gb + PrepGate::kDq;
+        const float *dkk_s = gb + PrepGate::kDkk, *bg_s = gb + PrepGate::kBg;
         wait_all(tma_bar, tma_phase);
         tma_phase ^= 1;
         psync();
         if (*abort_s) break;
-        // ---- [K; Q] K^T, the two K halves from two issuing threads (it depends on
-        //      the tiles only, so it runs while the gates are prepared) ---------------
+        // ---- [K; Q] K^T, the two K halves from two issuing threads ----------------
         if (tid == 0 || tid == 64) {
             const int part = tid >> 6;
             tc_fence_after();
@@ -232,46 +285,8 @@ __device__ __forceinline__ void prep_pipeline(
             }
             mma_commit(g_bar);
         }
-        if (tid < 64 && desc[nxt * 4]) load_gates(desc[nxt * 4 + 1], desc[nxt * 4 + 2], desc[nxt * 4 + 3], al_n, bt_n);
-        if (warp == 0) {  // inclusive prefix sum of log alpha, 2 rows per lane
-            const float a0 = g_s[2 * lane], a1 = g_s[2 * lane + 1];
-            float s = a0 + a1;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, s, d);
-                if (lane >= d) s += y;
-            }
-            const float ex = s - (a0 + a1);
-            g_s[2 * lane] = ex + a0;
-            g_s[2 * lane + 1] = ex + a0 + a1;
-        }
-        if (tid < 64) {   // only warps 0 and 1 use the prefix sums before the next barrier
-            sync64();
-            const float gr = g_s[tid], gl = g_s[63];
-            dq_s[tid] = rev ? (tid > 0 ? __expf(g_s[tid - 1]) : 1.f) : __expf(gr);
-            dkk_s[tid] = __expf(gl - gr);
-            bg_s[tid] = beta_s[tid] * __expf(gr);
-            if (tid == 0) *ds_s = __expf(gl);
-            // Decay factors of the masks without an exponential per entry: for s in
-            // the 16-token block k, e^{g_r - g_s} = e^{g_r - g_16k} e^{g_16k - g_s}.
-            // On the entries the masks keep (16k <= s <= r) the first factor is at
-            // most 1 and the second at most e^(decay over 16 tokens), so both are
-            // finite whenever that decay stays below 80 (else: one exponential per
-            // entry).  (Scratch: the band buffer, unused until the inverse.)
-            const float gqr = rev ? (tid > 0 ? g_s[tid - 1] : 0.f) : gr;
-            Xsm[tid] = __expf(g_s[tid & ~15] - gr);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                Xsm[64 + tid * 4 + k] = __expf(gr - g_s[16 * k]);
-                Xsm[320 + tid * 4 + k] = __expf(gqr - g_s[16 * k]);
-            }
-            if (tid == 0) {
-                bool fast = true;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) fast = fast && (g_s[16 * k] - g_s[16 * k + 15] < 80.f);
-                reinterpret_cast<int *>(Xsm)[576] = fast ? 1 : 0;
-            }
-        }
+        if (warp == 4 && desc[nxt * 4])   // the next task's gates, made during this task's level 2
+            load_gates(desc[nxt * 4 + 1], desc[nxt * 4 + 2], desc[nxt * 4 + 3], al_n, bt_n);
         // the previous task's record stores must have read the staging areas; when
         // a chain runs alongside, wait for them to land and flag that record
         if (tid == 0) {
@@ -288,7 +303,7 @@ __device__ __forceinline__ void prep_pipeline(
         wait_all(g_bar, g_phase);
         g_phase ^= 1;
         tc_fence_after();
-        psync();  // gate vectors ready
+        psync();
         // ---- L (fp32, to shared), P (fp16 image, staged for a bulk store) and the
         //      key-norm term of the state map's bound --------------------------------
         {
@@ -307,13 +322,13 @@ __device__ __forceinline__ void prep_pipeline(
             const int fl = ln & 63;                      // forward row within the chunk
             const int r = rev ? 63 - fl : fl;            // processing row
             const int f0 = half * 32;                    // forward columns f0 .. f0+31
-            const bool fast = reinterpret_cast<const int *>(Xsm)[576] != 0;   // task-uniform
-            const float *facs = Xsm;                                       // e^{g_16k - g_s}
+            const bool fast = reinterpret_cast<const int *>(gb)[PrepGate::kFast] != 0;   // task-uniform
+            const float *facs = gb + PrepGate::kFacs;                                  // e^{g_16k - g_s}
             // the 16-token blocks of this thread's 32 columns: first 16, last 16
             const int kA = rev ? 3 - (f0 >> 4) : (f0 >> 4), kB = rev ? 2 - (f0 >> 4) : (f0 >> 4) + 1;
             if (ln < 64) {
                 const float br = beta_s[r], gr = g_s[r];
-                const float eA = br * Xsm[64 + r * 4 + kA], eB = br * Xsm[64 + r * 4 + kB];
+                const float eA = br * __expf(gr - g_s[16 * kA]), eB = br * __expf(gr - g_s[16 * kB]);
                 // (the decay test is task-uniform: one loop or the other runs)
                 if (fast) {
 #pragma unroll
@@ -339,7 +354,7 @@ __device__ __forceinline__ void prep_pipeline(
                 }
             } else {
                 const float gq = rev ? (r > 0 ? g_s[r - 1] : 0.f) : g_s[r];
-                const float eA = Xsm[320 + r * 4 + kA], eB = Xsm[320 + r * 4 + kB];
+                const float eA = __expf(gq - g_s[16 * kA]), eB = __expf(gq - g_s[16 * kB]);
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     float v[8];
@@ -374,7 +389,7 @@ __device__ __forceinline__ void prep_pipeline(
             bulk_store(rec + RC::kP, smem + SM::kT1, 8192);
             bulk_commit_group();
             lb[(size_t)(dir * nbh + bh) * nC + c] = g_s[63] + kf_s[0] + kf_s[1];
-            rgate_s[0] = *ds_s;
+            rgate_s[0] = gb[PrepGate::kDs];
             rgate_s[1] = rgate_s[2] = rgate_s[3] = 0.f;
         }
         // ---- T = (I + L)^{-1}, blocked 16 x 16 (processing order); meanwhile the
@@ -446,6 +461,10 @@ __device__ __forceinline__ void prep_pipeline(
             }
             Tsm[a * 65 + bc] = -y00; Tsm[a * 65 + bc + 1] = -y01;
             Tsm[(a + 1) * 65 + bc] = -y10; Tsm[(a + 1) * 65 + bc + 1] = -y11;
+        } else if (warp == 4 && desc[nxt * 4]) {
+            // the next task's gates, into the other buffer (the last task that
+            // used it is done)
+            make_gates(gate_s + nxt * PrepGate::kFloats, al_n, bt_n, desc[nxt * 4 + 1] != 0);
         }
         psync();
         // level 3, X = L_[32:64, 0:32] T_[0:32, 0:32] (32 x 32, fp32, stride 33) in the
