@@ -136,8 +136,8 @@ def kernel_algorithmic_bytes(name, w, out_bytes=4):
 # launch processes.  Keyed by (kernel, workload); absent means not captured
 # for this kernel as it stands.
 MEASURED_TRAFFIC_PER_TOKEN_HEAD = {
-    ("tc_prep", "skewed"): (203.614976e6 + 265.897216e6) / (4 * 32 * 2048),   # prep_kernel<128>, T = 2048
-    ("tc_chain", "skewed"): (302.58432e6 + 105.378048e6) / (4 * 32 * 2048),   # chain_kernel<128, float>, T = 2048
+    ("tc_prep", "skewed"): (203.651072e6 + 248.647424e6) / (4 * 32 * 2048),   # prep_kernel<128>, T = 2048
+    ("tc_chain", "skewed"): (302.596608e6 + 105.210368e6) / (4 * 32 * 2048),   # chain_kernel<128, float>, T = 2048
 }
 
 

@@ -66,8 +66,7 @@ struct PrepSmem {
 
 constexpr int kPrepThreads = 256;
 constexpr int kPrepCtasPerSm = 2;
-constexpr uint32_t kPrepColG = 0;      // 128 lanes x 64, first K half (dead before W is written)
-constexpr uint32_t kPrepColG2 = 64;    // second K half
+constexpr uint32_t kPrepColG = 0;      // Gram [K; Q] K^T, 128 lanes x 64 (dead before W is written)
 constexpr uint32_t kPrepColW = 0;      // M=64 x 128
 constexpr uint32_t kPrepColU = 128;    // M=64 x DV
 constexpr uint32_t kPrepTmemCols = 256;
@@ -118,7 +117,7 @@ __device__ __forceinline__ void prep_pipeline(
     float *rgate_s = reinterpret_cast<float *>(smem + SM::kMisc + 16); // [4] record gate (ds)
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + SM::kBar);
     uint64_t *mma_bar = tma_bar + 1;
-    uint64_t *g_bar = tma_bar + 2;     // the two K halves of the Gram product
+    uint64_t *g_bar = tma_bar + 2;     // the Gram product
     volatile int *abort_s = reinterpret_cast<volatile int *>(smem + SM::kCtl + 4);
 
     const int tid = ptid, warp = tid >> 5, lane = tid & 31;
@@ -133,7 +132,7 @@ __device__ __forceinline__ void prep_pipeline(
     if (tid == 0) {
         mbar_init(tma_bar, 1);
         mbar_init(mma_bar, 1);
-        mbar_init(g_bar, 2);
+        mbar_init(g_bar, 1);
         fence_mbar_init();
         *abort_s = 0;
         prefetch_tensormap(tm_k);
@@ -273,15 +272,14 @@ __device__ __forceinline__ void prep_pipeline(
         tma_phase ^= 1;
         psync();
         if (*abort_s) break;
-        // ---- [K; Q] K^T, the two K halves from two issuing threads ----------------
-        if (tid == 0 || tid == 64) {
-            const int part = tid >> 6;
+        // ---- [K; Q] K^T (one accumulator, the two 64-column blocks of d_k in turn) ---
+        if (tid == 0) {
             tc_fence_after();
             constexpr uint32_t id = idesc(128, 64, 1, 0, 0);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t a = st_addr + part * 16384 + k * 32;
-                mma_bf16(tmem + (part ? kPrepColG2 : kPrepColG), sdesc_sw128(a), sdesc_sw128(a), id, k > 0);
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t a = st_addr + (k >> 2) * 16384 + (k & 3) * 32;
+                mma_bf16(tmem + kPrepColG, sdesc_sw128(a), sdesc_sw128(a), id, k > 0);
             }
             mma_commit(g_bar);
         }
@@ -308,80 +306,79 @@ __device__ __forceinline__ void prep_pipeline(
         //      key-norm term of the state map's bound --------------------------------
         {
             float G[32];
-            {
-                float G2[32];
-                tmem_ld16(tmem + lane_base + kPrepColG + half * 32, G);
-                tmem_ld16(tmem + lane_base + kPrepColG + half * 32 + 16, G + 16);
-                tmem_ld16(tmem + lane_base + kPrepColG2 + half * 32, G2);
-                tmem_ld16(tmem + lane_base + kPrepColG2 + half * 32 + 16, G2 + 16);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) G[e] += G2[e];
-            }
-            const int ln = quarter * 32 + lane;          // TMEM lane = Gram row
-            const int fl = ln & 63;                      // forward row within the chunk
-            const int r = rev ? 63 - fl : fl;            // processing row
-            const int f0 = half * 32;                    // forward columns f0 .. f0+31
-            const bool fast = reinterpret_cast<const int *>(gb)[PrepGate::kFast] != 0;   // task-uniform
-            const float *facs = gb + PrepGate::kFacs;                                  // e^{g_16k - g_s}
-            // the 16-token blocks of this thread's 32 columns: first 16, last 16
-            const int kA = rev ? 3 - (f0 >> 4) : (f0 >> 4), kB = rev ? 2 - (f0 >> 4) : (f0 >> 4) + 1;
-            if (ln < 64) {
-                const float br = beta_s[r], gr = g_s[r];
-                const float eA = br * __expf(gr - g_s[16 * kA]), eB = br * __expf(gr - g_s[16 * kB]);
-                // (the decay test is task-uniform: one loop or the other runs)
-                if (fast) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int s = rev ? 63 - (f0 + e) : f0 + e;
-                        Lsm[r * 65 + s] = s < r ? (e < 16 ? eA : eB) * facs[s] * G[e] : 0.f;
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int s = rev ? 63 - (f0 + e) : f0 + e;
-                        Lsm[r * 65 + s] = s < r ? br * __expf(gr - g_s[s]) * G[e] : 0.f;
-                    }
-                }
-                if (half == (fl >> 5)) {   // warps 0 and 5 hold the diagonal of rows 0-31 / 32-63
-                    float kk = 0.f;        // |k_r|^2: the Gram's diagonal, column fl - f0 = lane
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) kk = e == lane ? G[e] : kk;
-                    float term = __logf(fmaxf(1.f, fabsf(1.f - br * kk)));
-#pragma unroll
-                    for (int d = 16; d > 0; d >>= 1) term += __shfl_xor_sync(0xffffffffu, term, d);
-                    if (lane == 0) kf_s[half] = term;
-                }
-            } else {
-                const float gq = rev ? (r > 0 ? g_s[r - 1] : 0.f) : g_s[r];
-                const float eA = __expf(gq - g_s[16 * kA]), eB = __expf(gq - g_s[16 * kB]);
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float v[8];
+            tmem_ld16(tmem + lane_base + kPrepColG + half * 32, G);
+            tmem_ld16(tmem + lane_base + kPrepColG + half * 32 + 16, G + 16);
+            tmem_wait_ld();
+            // the mask code once per direction, so that the column order of every
+            // entry (forward or mirrored) is a compile-time constant
+            auto mask = [&](auto rv_c) {
+                constexpr bool rev = decltype(rv_c)::value;   // (shadows the task flag)
+                const int ln = quarter * 32 + lane;          // TMEM lane = Gram row
+                const int fl = ln & 63;                      // forward row within the chunk
+                const int r = rev ? 63 - fl : fl;            // processing row
+                const int f0 = half * 32;                    // forward columns f0 .. f0+31
+                const bool fast = reinterpret_cast<const int *>(gb)[PrepGate::kFast] != 0;   // task-uniform
+                const float *facs = gb + PrepGate::kFacs;                                  // e^{g_16k - g_s}
+                // the 16-token blocks of this thread's 32 columns: first 16, last 16
+                const int kA = rev ? 3 - (f0 >> 4) : (f0 >> 4), kB = rev ? 2 - (f0 >> 4) : (f0 >> 4) + 1;
+                if (ln < 64) {
+                    const float br = beta_s[r], gr = g_s[r];
+                    const float eA = br * __expf(gr - g_s[16 * kA]), eB = br * __expf(gr - g_s[16 * kB]);
+                    // (the decay test is task-uniform: one loop or the other runs)
                     if (fast) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int f = f0 + cc * 8 + e;
-                            const int s = rev ? 63 - f : f;
-                            const bool keep = rev ? (s < r) : (s <= r);
-                            v[e] = keep ? (cc < 2 ? eA : eB) * facs[s] * G[cc * 8 + e] : 0.f;
+                        for (int e = 0; e < 32; ++e) {
+                            const int s = rev ? 63 - (f0 + e) : f0 + e;
+                            Lsm[r * 65 + s] = s < r ? (e < 16 ? eA : eB) * facs[s] * G[e] : 0.f;
                         }
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int f = f0 + cc * 8 + e;
-                            const int s = rev ? 63 - f : f;
-                            const bool keep = rev ? (s < r) : (s <= r);
-                            v[e] = keep ? __expf(gq - g_s[s]) * G[cc * 8 + e] : 0.f;
+                        for (int e = 0; e < 32; ++e) {
+                            const int s = rev ? 63 - (f0 + e) : f0 + e;
+                            Lsm[r * 65 + s] = s < r ? br * __expf(gr - g_s[s]) * G[e] : 0.f;
                         }
                     }
-                    uint4 p;
-                    p.x = pack_f16(v[0], v[1]); p.y = pack_f16(v[2], v[3]);
-                    p.z = pack_f16(v[4], v[5]); p.w = pack_f16(v[6], v[7]);
-                    *reinterpret_cast<uint4 *>(smem + SM::kT1 + sw128(fl, f0 + cc * 8, 0)) = p;
+                    if (half == (fl >> 5)) {   // warps 0 and 5 hold the diagonal of rows 0-31 / 32-63
+                        float kk = 0.f;        // |k_r|^2: the Gram's diagonal, column fl - f0 = lane
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) kk = e == lane ? G[e] : kk;
+                        float term = __logf(fmaxf(1.f, fabsf(1.f - br * kk)));
+#pragma unroll
+                        for (int d = 16; d > 0; d >>= 1) term += __shfl_xor_sync(0xffffffffu, term, d);
+                        if (lane == 0) kf_s[half] = term;
+                    }
+                } else {
+                    const float gq = rev ? (r > 0 ? g_s[r - 1] : 0.f) : g_s[r];
+                    const float eA = __expf(gq - g_s[16 * kA]), eB = __expf(gq - g_s[16 * kB]);
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float v[8];
+                        if (fast) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int f = f0 + cc * 8 + e;
+                                const int s = rev ? 63 - f : f;
+                                const bool keep = rev ? (s < r) : (s <= r);
+                                v[e] = keep ? (cc < 2 ? eA : eB) * facs[s] * G[cc * 8 + e] : 0.f;
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int f = f0 + cc * 8 + e;
+                                const int s = rev ? 63 - f : f;
+                                const bool keep = rev ? (s < r) : (s <= r);
+                                v[e] = keep ? __expf(gq - g_s[s]) * G[cc * 8 + e] : 0.f;
+                            }
+                        }
+                        uint4 p;
+                        p.x = pack_f16(v[0], v[1]); p.y = pack_f16(v[2], v[3]);
+                        p.z = pack_f16(v[4], v[5]); p.w = pack_f16(v[6], v[7]);
+                        *reinterpret_cast<uint4 *>(smem + SM::kT1 + sw128(fl, f0 + cc * 8, 0)) = p;
+                    }
+                    fence_async_shared();
                 }
-                fence_async_shared();
-            }
+            };
+            if (rev) mask(std::true_type{}); else mask(std::false_type{});
         }
         tc_fence_before();
         psync();
