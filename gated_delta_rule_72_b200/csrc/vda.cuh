@@ -16,7 +16,7 @@
 // Four steps:
 //   vda_gram    (frame x head, fully parallel)  A_f and B_f
 //   vda_factor  (frame x head, fully parallel)  P_f = (I + A_f)^{-1} by a
-//               Cholesky factorisation: none of it depends on the state
+//               blocked Cholesky factorisation: none of it depends on the state
 //   vda_chain   (head x direction x 32 state columns, sequential over frames)
 //               S <- P_f (alpha_f S + B_f), the slice of the state in shared
 //               memory; stores the state each frame's readout uses
@@ -123,109 +123,239 @@ vda_gram_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const floa
 
 // ---------------------------------------------------------------------------
 // Factor (frame x head, fully parallel: nothing here depends on the state):
-// P_f = (I + A_f)^{-1}, written over A_f.
-//
-// M = I + A_f = L L^T (Cholesky, right-looking, one barrier per column: step
-// j reads the pivot and column j of the lower triangle, writes L's column j
-// transposed into the upper triangle (row j, which no later step reads or
-// writes) and subtracts the column's outer product from the trailing lower
-// triangle; warp w takes the rows i = w mod 16, its lanes the columns).
-// Then L Y = I and L^T P = Y with no block barrier: each warp owns 8
-// right-hand-side columns, each column's 4 lanes split its rows (i = g mod
-// 4), so a step only involves lanes of one warp.
+// P_f = (I + A_f)^{-1}, written over A_f, on blocks of 32 x 32 (NB = DK / 32
+// block rows), fp32:
+//   1. M = I + A_f = L L^T, a blocked right-looking Cholesky.  Per block
+//      column: warp 0 factors the diagonal block in registers, a thread per
+//      row below it solves for the panel L_ip (forward substitution against
+//      L_pp), and all threads apply the trailing update M_ij -= L_ip L_jp^T.
+//      Three barriers per block column instead of one per column.
+//   2. Y = L^{-1}: the diagonal blocks' inverses (a warp each), then
+//      recursive doubling over the blocks: Y_10 = -Y_11 (L_10 Y_00) in each
+//      pair of blocks, then the same on the pair of pairs.
+//   3. P = Y^T Y (P_ij = sum over k >= max(i, j) of Y_ki Y_kj).
 // ---------------------------------------------------------------------------
 template <int DK, int DV>
 struct FactorSmem {
-    static constexpr int kW = DK;                          // right-hand sides: I
-    static constexpr int kLdM = DK + 1;                    // odd stride: column walks are conflict-free
-    static constexpr int kLdX = kW + 8;                    // 4 row groups of a column on 4 bank groups
+    static constexpr int kLdM = DK + 1;                    // L: odd stride, column walks conflict-free
+    static constexpr int kLdY = DK + 4;                    // Y = L^{-1}: rows 16-byte aligned
+    static constexpr int kLdX = DK / 2 + 1;                // doubling scratch
     static constexpr int kM = 0;
-    static constexpr int kX = kM + DK * kLdM * 4;
-    static constexpr int kD = kX + DK * kLdX * 4;          // 1 / diagonal of L
+    static constexpr int kY = kM + (DK * kLdM * 4 + 15) / 16 * 16;
+    static constexpr int kX = kY + DK * kLdY * 4;
+    static constexpr int kD = kX + (DK / 2) * kLdX * 4;    // 1 / diagonal of L
     static constexpr int kBytes = kD + DK * 4;
 };
+
+// Warp-level pieces of the factor (p0: first row of a 32 x 32 diagonal
+// block; runtime, so that one copy of this straight-line code serves every
+// block).
+//
+// Cholesky of the diagonal block in registers: lane i holds row i, column j's
+// entries reach the other lanes by shuffles.  Entries right of the diagonal
+// (k > lane) take part in the arithmetic but only ever feed entries right of
+// the diagonal, and are written as zeros.  rd[p0 + j] = 1 / L_jj.
+__device__ __forceinline__ void chol_diag_block(float *M, float *rd, int LM, int p0, int lane) {
+    float a[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) a[k] = M[(p0 + lane) * LM + p0 + k];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const float r = rsqrtf(__shfl_sync(0xffffffffu, a[j], j));
+        if (lane == j) rd[p0 + j] = r;
+        a[j] *= r;
+#pragma unroll
+        for (int k = j + 1; k < 32; ++k) a[k] = fmaf(-a[j], __shfl_sync(0xffffffffu, a[j], k), a[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 32; ++k) M[(p0 + lane) * LM + p0 + k] = k <= lane ? a[k] : 0.f;
+}
+
+// Panel row `row` below the diagonal block: x L_pp^T = m by forward
+// substitution, in place (L_pp read with every lane at the same address).
+__device__ __forceinline__ void chol_panel_row(float *M, const float *rd, int LM, int p0, int row) {
+    float x[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) x[k] = M[row * LM + p0 + k];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        float acc = x[k];
+#pragma unroll
+        for (int j = 0; j < k; ++j) acc = fmaf(-x[j], M[(p0 + k) * LM + p0 + j], acc);
+        x[k] = acc * rd[p0 + k];
+    }
+#pragma unroll
+    for (int k = 0; k < 32; ++k) M[row * LM + p0 + k] = x[k];
+}
+
+// Inverse of the diagonal block: lane c computes column c,
+// y_i = (delta_ic - sum_{k<i} L_ik y_k) / L_ii (zero above the diagonal by itself).
+__device__ __forceinline__ void diag_block_inverse(const float *M, const float *rd, float *Y, int LM, int LY,
+                                                   int p0, int lane) {
+    float y[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        float acc = i == lane ? 1.f : 0.f;
+#pragma unroll
+        for (int k = 0; k < i; ++k) acc = fmaf(-M[(p0 + i) * LM + p0 + k], y[k], acc);
+        y[i] = acc * rd[p0 + i];
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) Y[(p0 + i) * LY + p0 + lane] = y[i];
+}
+
+// Trailing update after block column p0: M_ij -= sum_k L_ik L_jk over the R x R
+// square below and right of the panel (only its lower triangle is used
+// later).  Thread rows ti + 32 a, columns tj + 16 b.
+template <int DK, int R>
+__device__ __forceinline__ void chol_trailing(float *M, int p0, int tid) {
+    constexpr int LM = DK + 1, NA = R / 32, NBc = R / 16;
+    const int ti = tid & 31, tj = tid >> 5, base = p0 + 32;
+    float acc[NA][NBc];
+#pragma unroll
+    for (int x = 0; x < NA; ++x)
+#pragma unroll
+        for (int z = 0; z < NBc; ++z) acc[x][z] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < 32; ++k) {
+        float li[NA], lj[NBc];
+#pragma unroll
+        for (int x = 0; x < NA; ++x) li[x] = M[(base + ti + 32 * x) * LM + p0 + k];
+#pragma unroll
+        for (int z = 0; z < NBc; ++z) lj[z] = M[(base + tj + 16 * z) * LM + p0 + k];
+#pragma unroll
+        for (int x = 0; x < NA; ++x)
+#pragma unroll
+            for (int z = 0; z < NBc; ++z) acc[x][z] = fmaf(li[x], lj[z], acc[x][z]);
+    }
+#pragma unroll
+    for (int x = 0; x < NA; ++x)
+#pragma unroll
+        for (int z = 0; z < NBc; ++z) M[(base + ti + 32 * x) * LM + base + tj + 16 * z] -= acc[x][z];
+}
+
+// One level of the recursive doubling for Y = L^{-1}: for every pair of
+// adjacent diagonal blocks of size S (bottom block rows [r0, r0+S), top
+// [r0-S, r0)), Y_bt = -Y_bb (L_bt Y_tt).  Each thread a 2 x 2 tile of the
+// products; X is the scratch for L_bt Y_tt.
+template <int DK, int S>
+__device__ __forceinline__ void inverse_level(const float *M, float *Y, float *X, int tid) {
+    constexpr int LM = DK + 1, LY = DK + 4, LX = DK / 2 + 1;
+    constexpr int NPAIR = DK / (2 * S), TILES = (S / 2) * (S / 2);      // 2 x 2 tiles per pair
+    static_assert(NPAIR * S <= DK / 2, "scratch rows");
+    for (int u = tid; u < NPAIR * TILES; u += kChainThreads) {   // X = L_bt Y_tt (Y_tt lower)
+        const int pr = u / TILES, t = u % TILES, i = 2 * (t / (S / 2)), j = 2 * (t % (S / 2));
+        const int top = 2 * S * pr, bot = top + S;
+        float *Xp = X + (pr * S) * LX;
+        float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < S; ++k) {
+            const float l0 = M[(bot + i) * LM + top + k], l1 = M[(bot + i + 1) * LM + top + k];
+            const float y0 = Y[(top + k) * LY + top + j], y1 = Y[(top + k) * LY + top + j + 1];
+            x00 = fmaf(l0, y0, x00); x01 = fmaf(l0, y1, x01);
+            x10 = fmaf(l1, y0, x10); x11 = fmaf(l1, y1, x11);
+        }
+        Xp[i * LX + j] = x00; Xp[i * LX + j + 1] = x01;
+        Xp[(i + 1) * LX + j] = x10; Xp[(i + 1) * LX + j + 1] = x11;
+    }
+    __syncthreads();
+    for (int u = tid; u < NPAIR * TILES; u += kChainThreads) {   // Y_bt = -Y_bb X (Y_bb lower)
+        const int pr = u / TILES, t = u % TILES, i = 2 * (t / (S / 2)), j = 2 * (t % (S / 2));
+        const int top = 2 * S * pr, bot = top + S;
+        const float *Xp = X + (pr * S) * LX;
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < S; ++k) {
+            const float a0 = Y[(bot + i) * LY + bot + k], a1 = Y[(bot + i + 1) * LY + bot + k];
+            const float x0 = Xp[k * LX + j], x1 = Xp[k * LX + j + 1];
+            y00 = fmaf(a0, x0, y00); y01 = fmaf(a0, x1, y01);
+            y10 = fmaf(a1, x0, y10); y11 = fmaf(a1, x1, y11);
+        }
+        Y[(bot + i) * LY + top + j] = -y00; Y[(bot + i) * LY + top + j + 1] = -y01;
+        Y[(bot + i + 1) * LY + top + j] = -y10; Y[(bot + i + 1) * LY + top + j + 1] = -y11;
+    }
+    __syncthreads();
+}
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kChainThreads)
 vda_factor_kernel(float *__restrict__ A)
 {
     using SM = FactorSmem<DK, DV>;
-    constexpr int LD = SM::kLdM, LX = SM::kLdX, W = SM::kW;
-    constexpr int NW = kChainThreads / 32;
-    static_assert(W % 8 == 0, "right-hand-side columns in groups of 8 (warp-uniform loop bounds)");
+    constexpr int LM = SM::kLdM, LY = SM::kLdY, NB = DK / 32;
+    static_assert(DK == 64 || DK == 128, "d_k of the factor");
     extern __shared__ __align__(16) unsigned char fsm[];
     float *M = reinterpret_cast<float *>(fsm + SM::kM);
+    float *Y = reinterpret_cast<float *>(fsm + SM::kY);
     float *X = reinterpret_cast<float *>(fsm + SM::kX);
-    float *rdL = reinterpret_cast<float *>(fsm + SM::kD);
+    float *rd = reinterpret_cast<float *>(fsm + SM::kD);
     const size_t fh = (size_t)blockIdx.x * gridDim.y + blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float *Af = A + fh * DK * DK;
     for (int e = tid; e < DK * DK; e += kChainThreads) {
         const int i = e / DK, j = e % DK;
-        M[i * LD + j] = Af[e] + (i == j ? 1.f : 0.f);
-        X[i * LX + j] = i == j ? 1.f : 0.f;
+        M[i * LM + j] = Af[e] + (i == j ? 1.f : 0.f);
+        Y[i * LY + j] = 0.f;
     }
     __syncthreads();
-    // ---- Cholesky
-    for (int j = 0; j < DK; ++j) {
-        const float piv = M[j * LD + j];
-        const float r = rsqrtf(piv), r2 = r * r;
-        for (int i = j + 1 + ((warp - (j + 1)) & (NW - 1)); i < DK; i += NW) {
-            const float mij = M[i * LD + j];
-            if (lane == 0) M[j * LD + i] = mij * r;        // L[i][j], kept at (j, i)
-            const float fct = mij * r2;
-            int cc = j + 1 + lane;
-            for (; cc + 96 <= i; cc += 128) {              // four columns loaded before any store
-                float lc[4], m[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    lc[q] = M[(cc + 32 * q) * LD + j];
-                    m[q] = M[i * LD + cc + 32 * q];
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) M[i * LD + cc + 32 * q] = fmaf(-fct, lc[q], m[q]);
-            }
-            for (; cc <= i; cc += 32) M[i * LD + cc] = fmaf(-fct, M[cc * LD + j], M[i * LD + cc]);
-        }
-        if (tid == 0) rdL[j] = r;                          // 1 / L[j][j]
+    // ---- 1. Cholesky, block column by block column: the diagonal block (warp
+    //      0), the panel below it (a thread per row), the trailing update (all)
+#pragma unroll 1
+    for (int p = 0; p < NB; ++p) {
+        const int p0 = 32 * p, R = DK - p0 - 32;
+        if (warp == 0) chol_diag_block(M, rd, LM, p0, lane);
+        __syncthreads();
+        if (R == 0) break;
+        if (tid < R) chol_panel_row(M, rd, LM, p0, p0 + 32 + tid);
+        __syncthreads();
+        if (R == DK - 32) chol_trailing<DK, DK - 32>(M, p0, tid);
+        else if (R == DK - 64) chol_trailing<DK, (DK > 64 ? DK - 64 : 32)>(M, p0, tid);
+        else chol_trailing<DK, 32>(M, p0, tid);
         __syncthreads();
     }
-    // ---- L Y = I, then L^T P = Y, column by column inside each warp.
-    // A step's row updates are independent: four rows are loaded before any is
-    // stored, so their shared-memory latencies overlap.
-    const int g = lane >> 3;
-    auto update_rows = [&](int i, int i_end, int c, float y, int lstride, int loff) {
-        // X[i][c] -= L * y for rows i, i+4, ... < i_end; L of row i at M[i*lstride + loff]
-        for (; i + 12 < i_end; i += 16) {
-            float l[4], x[4];
+    // ---- 2. Y = L^{-1}: the diagonal blocks (a warp each), then recursive
+    //      doubling on pairs of 32-blocks and (for d_k = 128) of 64-blocks
+    if (warp < NB) diag_block_inverse(M, rd, Y, LM, LY, 32 * warp, lane);
+    __syncthreads();
+    inverse_level<DK, 32>(M, Y, X, tid);
+    if constexpr (NB == 4) inverse_level<DK, 64>(M, Y, X, tid);
+    // ---- 3. P = Y^T Y.  Warp w owns row tiles of 4 rows (w and, for d_k = 128,
+    //      31 - w, so that every warp has the same number of terms); lane l
+    //      columns CW l .. CW l + CW - 1.  Terms k < the tile's first row are
+    //      zero (Y lower triangular) and skipped.
+    constexpr int CW = DK / 32;
+    constexpr int NT = DK / 64;                       // row tiles per warp
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                l[q] = M[(i + 4 * q) * lstride + loff];
-                x[q] = X[(i + 4 * q) * LX + c];
+    for (int tt = 0; tt < NT; ++tt) {
+        const int i0 = 4 * (tt == 0 ? warp : (DK / 4 - 1 - warp));
+        float acc[4][CW];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < CW; ++c) acc[r][c] = 0.f;
+        for (int k = i0; k < DK; ++k) {
+            const float4 yi = *reinterpret_cast<const float4 *>(Y + k * LY + i0);
+            float yj[CW];
+            if constexpr (CW == 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(Y + k * LY + CW * lane);
+                yj[0] = v.x; yj[1] = v.y; yj[2] = v.z; yj[3] = v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2 *>(Y + k * LY + CW * lane);
+                yj[0] = v.x; yj[1] = v.y;
             }
+            const float yr[4] = {yi.x, yi.y, yi.z, yi.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) X[(i + 4 * q) * LX + c] = fmaf(-l[q], y, x[q]);
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < CW; ++c) acc[r][c] = fmaf(yr[r], yj[c], acc[r][c]);
         }
-        for (; i < i_end; i += 4) X[i * LX + c] = fmaf(-M[i * lstride + loff], y, X[i * LX + c]);
-    };
-    for (int c = warp * 8 + (lane & 7); c < W; c += NW * 8) {
-        for (int j = 0; j < DK; ++j) {
-            const float y = X[j * LX + c] * rdL[j];
-            __syncwarp();
-            if ((j & 3) == g) X[j * LX + c] = y;
-            update_rows(j + 1 + ((g - (j + 1)) & 3), DK, c, y, 1, j * LD);    // L[i][j] at (j, i)
-            __syncwarp();
-        }
-        for (int j = DK - 1; j >= 0; --j) {
-            const float y = X[j * LX + c] * rdL[j];
-            __syncwarp();
-            if ((j & 3) == g) X[j * LX + c] = y;
-            update_rows(g, j, c, y, LD, j);                                   // L[j][i] at (i, j)
-            __syncwarp();
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            float *dst = Af + (size_t)(i0 + r) * DK + CW * lane;
+            if constexpr (CW == 4) *reinterpret_cast<float4 *>(dst) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+            else *reinterpret_cast<float2 *>(dst) = make_float2(acc[r][0], acc[r][1]);
         }
     }
-    __syncthreads();
-    for (int e = tid; e < DK * DK; e += kChainThreads) Af[e] = X[(e / DK) * LX + e % DK];
 }
 
 // ---------------------------------------------------------------------------
