@@ -365,7 +365,9 @@ vda_factor_kernel(float *__restrict__ A)
 // goes to `st` ([dir][F][B*H][DK][DV]): the causal direction stores S_f, the
 // reverse one R_{f+1} (before the frame is written), as fp32 or (kImage) as
 // the tensor-core readout's operand image.  Thread tile 4 rows x 2 columns;
-// P_f (symmetric: row k of P is column k) is staged in shared memory.
+// P_f (symmetric: row k of P is column k) and the slice of B_f are staged in
+// shared memory, double-buffered: the next frame's are fetched (cp.async)
+// while this frame's product runs.
 // ---------------------------------------------------------------------------
 constexpr int kSlice = 32;
 
@@ -395,10 +397,21 @@ __device__ __forceinline__ void store_image_row8(unsigned char *img, int i, int 
 
 template <int DK, int DV>
 struct ChainSmem {
-    static constexpr int kP = 0;                           // [DK][DK]
-    static constexpr int kS = kP + DK * DK * 4;            // [DK][kSlice]
+    static constexpr int kP = 0;                           // 2 x [DK][DK]
+    static constexpr int kB = kP + 2 * DK * DK * 4;        // 2 x [DK][kSlice]
+    static constexpr int kS = kB + 2 * DK * kSlice * 4;    // [DK][kSlice]
     static constexpr int kBytes = kS + DK * kSlice * 4;
 };
+
+// 16-byte asynchronous copy global -> shared (completion by cp_async_wait_all)
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 template <int DK, int DV, bool kImage>
 __global__ void __launch_bounds__(kChainThreads)
@@ -413,6 +426,7 @@ vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ Bm, cons
     static_assert(kTiles <= kChainThreads && DV % kSlice == 0, "thread tiles");
     extern __shared__ __align__(16) unsigned char csm[];
     float *Ps = reinterpret_cast<float *>(csm + SM::kP);
+    float *Bs = reinterpret_cast<float *>(csm + SM::kB);
     float *S = reinterpret_cast<float *>(csm + SM::kS);
     const int bh = blockIdx.x, nbh = gridDim.x, dir = blockIdx.y, j0 = blockIdx.z * kSlice;
     const int b = bh / H, h = bh % H;
@@ -441,20 +455,40 @@ vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ Bm, cons
         }
     };
 
+    // the frame of step `stp`: P_f and the slice of B_f into buffer `buf`
+    auto fetch = [&](int stp, int buf) {
+        const int f = dir ? F - 1 - stp : stp;
+        const size_t fh = (size_t)f * nbh + bh;
+        const float *Pg = P + fh * DK * DK;
+        float *Pd = Ps + buf * DK * DK;
+        for (int e = tid * 4; e < DK * DK; e += kChainThreads * 4) cp_async16(Pd + e, Pg + e);
+        float *Bd = Bs + buf * DK * kSlice;
+        for (int e = tid * 4; e < DK * kSlice; e += kChainThreads * 4)
+            cp_async16(Bd + e, Bm + fh * sdim + (size_t)(e / kSlice) * DV + j0 + e % kSlice);
+        cp_async_commit();
+    };
+    auto alpha_of = [&](int stp) { return alpha_f[((size_t)b * F + (dir ? F - 1 - stp : stp)) * H + h]; };
+    fetch(0, 0);
+    float a_next = alpha_of(0);
+
     for (int step = 0; step < F; ++step) {
         const int f = dir ? F - 1 - step : step;
         const size_t fh = (size_t)f * nbh + bh;
-        const float a = alpha_f[((size_t)b * F + f) * H + h];
+        const float a = a_next;
+        const int buf = step & 1;
+        const float *Pf = Ps + buf * DK * DK, *Bf = Bs + buf * DK * kSlice;
         float *dst = st + ((size_t)dir * F * nbh + fh) * sdim;
-        __syncthreads();                                   // S complete, P free
-        if (dir) store_state(dst);                         // the reverse readout of frame f reads R_{f+1}
-        for (int e = tid * 4; e < DK * DK; e += kChainThreads * 4)
-            *reinterpret_cast<float4 *>(Ps + e) = *reinterpret_cast<const float4 *>(P + fh * DK * DK + e);
-        __syncthreads();
-        for (int e = tid; e < DK * kSlice; e += kChainThreads) {   // S <- alpha S + B
-            const int i = e / kSlice, c = e % kSlice;
-            S[e] = fmaf(a, S[e], Bm[fh * sdim + (size_t)i * DV + j0 + c]);
+        cp_async_wait_all();
+        __syncthreads();                                   // P_f, B_f landed; S complete; the other buffers free
+        if (step + 1 < F) {
+            fetch(step + 1, buf ^ 1);
+            a_next = alpha_of(step + 1);
         }
+        if (dir) {                                         // the reverse readout of frame f reads R_{f+1}
+            store_state(dst);
+            __syncthreads();
+        }
+        for (int e = tid; e < DK * kSlice; e += kChainThreads) S[e] = fmaf(a, S[e], Bf[e]);   // S <- alpha S + B
         __syncthreads();
         float acc[TR][TCc];
         if (worker) {
@@ -464,7 +498,7 @@ vda_chain_kernel(const float *__restrict__ P, const float *__restrict__ Bm, cons
                 for (int cc = 0; cc < TCc; ++cc) acc[r][cc] = 0.f;
 #pragma unroll 8
             for (int kk = 0; kk < DK; ++kk) {
-                const float4 pv = *reinterpret_cast<const float4 *>(Ps + kk * DK + i0);   // P[i0..][kk]
+                const float4 pv = *reinterpret_cast<const float4 *>(Pf + kk * DK + i0);   // P[i0..][kk]
                 const float2 sv = *reinterpret_cast<const float2 *>(S + kk * kSlice + c0);
                 const float pa[TR] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
