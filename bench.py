@@ -97,10 +97,23 @@ def vda_kernel_flops(w):
     (2 dk^3); per frame and direction S <- P (a S + B) (2 dk^2 dv); the
     readout of the two summed states (2 dk dv per token)."""
     dk, dv, U = w.dk, w.dv, w.frame
-    return {"vda_gram": 2.0 * dk * (dk + dv),
-            "vda_factor": (dk ** 3 / 3.0 + 2.0 * dk ** 3) / U,
-            "vda_chain": 2 * 2.0 * dk * dk * dv / U,
-            "vda_readout": 2.0 * dk * dv}
+    f = {"vda_gram": 2.0 * dk * (dk + dv),
+         "vda_factor": (dk ** 3 / 3.0 + 2.0 * dk ** 3) / U,
+         "vda_chain": 2 * 2.0 * dk * dk * dv / U,
+         "vda_readout": 2.0 * dk * dv}
+    f["vda_gram_tc"], f["vda_readout_tc"] = f["vda_gram"], f["vda_readout"]
+    return f
+
+
+def vda_kernel_bytes(name, w, out_bytes=4):
+    """Algorithmic HBM bytes per token-head of the frame-wise operator's
+    streaming kernels: the Gram reads k, v and beta; the readout reads q and
+    the two directions' states of its frame (fp32-sized, per frame of U
+    tokens) and writes o."""
+    ib = 4 if w.dtype == "f32" else 2
+    if "gram" in name:
+        return ib * (w.dk + w.dv) + 4
+    return ib * w.dk + out_bytes * w.dv + 2 * 4 * w.dk * w.dv / w.frame
 
 
 # fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA/clk x 2 FLOP x 1.965 GHz
@@ -388,7 +401,11 @@ def roofline_of(w, ktimes, steps, units, peaks, peak_src):
     units_per_launch = units / launches_per_step
     bound = "tensor" if w.mode == "bidir" and "chain" not in name else "hbm"
     if w.mode == "vda":
-        bound = "alu"     # fp32 on the CUDA cores
+        # the factor and the chain are fp32 on the CUDA cores; the Gram and
+        # the readout stream their operands from HBM
+        bound = "hbm" if ("gram" in name or "readout" in name) else "alu"
+    nbytes = (lambda ob=4: vda_kernel_bytes(name, w, ob)) if w.mode == "vda" else \
+        (lambda ob=4: kernel_algorithmic_bytes(name, w, out_bytes=ob))
     extra = {}
     if bound == "alu":
         alg = vda_kernel_flops(w).get(name, 0.0) * units_per_launch
@@ -396,15 +413,15 @@ def roofline_of(w, ktimes, steps, units, peaks, peak_src):
         peak = FP32_ALU_TFLOPS
         unit = "TFLOP/s"
     elif bound == "hbm":
-        alg = kernel_algorithmic_bytes(name, w) * units_per_launch
+        alg = nbytes() * units_per_launch
         achieved = alg / (per_launch_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         unit = "GB/s"
         # the same kernel against the survey's byte count, o in bf16
-        alg16 = kernel_algorithmic_bytes(name, w, out_bytes=2) * units_per_launch
+        alg16 = nbytes(2) * units_per_launch
         extra = {"frac_bf16_out_bytes": alg16 / (per_launch_ms * 1e-3) / 1e9 / peak,
-                 "bytes_per_token_head": kernel_algorithmic_bytes(name, w),
-                 "bytes_per_token_head_bf16_out": kernel_algorithmic_bytes(name, w, out_bytes=2)}
+                 "bytes_per_token_head": nbytes(),
+                 "bytes_per_token_head_bf16_out": nbytes(2)}
     else:
         alg = flops_per_token_head(w) * units_per_launch
         achieved = alg / (per_launch_ms * 1e-3) / 1e12
