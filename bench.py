@@ -417,7 +417,7 @@ def roofline_of(w, ktimes, steps, units, peaks, peak_src):
         achieved = alg / (per_launch_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         unit = "GB/s"
-        # the same kernel against the survey's byte count, o in bf16
+        # the same kernel against the byte count with o in bf16 (the inputs' dtype)
         alg16 = nbytes(2) * units_per_launch
         extra = {"frac_bf16_out_bytes": alg16 / (per_launch_ms * 1e-3) / 1e9 / peak,
                  "bytes_per_token_head": nbytes(),
@@ -445,8 +445,8 @@ def roofline_of(w, ktimes, steps, units, peaks, peak_src):
 
 def step_roofline(w, ms, peaks):
     """The whole step against its roofline: bytes at HBM bandwidth vs FLOPs at
-    the tensor peak; bytes with o in fp32 (as written here) and in bf16 (the
-    survey's count)."""
+    the tensor peak; bytes with o in fp32 (as written here) and in bf16 (o in
+    the inputs' dtype)."""
     t_flop = w.token_heads * flops_per_token_head(w) / (peaks["bf16_tflops"] * 1e12)
     out = {}
     for key, ob in (("", 4), ("_bf16_out", 2)):
