@@ -295,18 +295,19 @@ std::atomic<int> g_chain_segments{-1};
 // prep would lag the chains and two launches do better.
 constexpr int kMinFusedPrepCtas = 32;
 // Fewest chunks per segment (a segment also walks back a few chunks first).
-constexpr int kMinSegChunks = 6;
+constexpr int kMinSegChunks = 4;
 // Tail positions of every segment the prep produces first (the next
 // segment's walk back reads them before anything else).
 constexpr int kTailFirst = 12;
 
 // Automatic plan (from B200 timings of the d = 128 workloads): when the walks
 // are long enough to cut, prep on every SM and then one wave of chain CTAs
-// (G = SMs / chains, at least 6 chunks per segment: a 32k-token causal scan
+// (G = SMs / chains, at least 4 chunks per segment: a 32k-token causal scan
 // of 12 heads 0.37 ms against 0.49 ms fused with 4 segments; bidirectional
 // 75k tokens of 20 heads 2.8 ms against 4.2 ms fused; 168 streaming calls of
-// 1,560 tokens and 16 heads 13.9 ms with 4 segments against 16.4 ms fused
-// with one); when they are not (short calls, or chains that fill the GPU),
+// 1,560 tokens and 16 heads 11.8 ms with 5 segments of 5 chunks, 13.3 ms with
+// 4 of 7, 12.6 ms with 9 of 3, 16.4 ms fused with one); when they are not
+// (short calls, or chains that fill the GPU),
 // one fused launch where the SMs allow it, whose prep runs beside the chains
 // so that the first chunk's record is ready early.  A forced segment count
 // takes the fused launch where the SMs allow it.

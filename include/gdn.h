@@ -214,7 +214,7 @@ GDN_API int gdn_set_short_call_tokens(int max_t);
  * gdn_set_chain_segments -- how many segments the tensor-core path cuts each
  * (b, h, direction) chunk walk into (sequence parallelism; bf16 inputs).
  * g < 1: automatic (the default): enough segments to occupy the SMs with one
- * wave of chain CTAs, at least 6 chunks each; g >= 1: g segments (at most one
+ * wave of chain CTAs, at least 4 chunks each; g >= 1: g segments (at most one
  * per chunk).
  * A segment other than the first starts from a zero state some chunks before
  * its first output, at the first chunk boundary where the 2-norm bound of the
